@@ -1,0 +1,175 @@
+"""fp64 CPU oracle for exact scaled-dot-product attention, forward and backward.
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module. The product path
+(``exact_attention_119_b200``) never imports it and shares no code with it.
+
+Sources (the web pages this build follows; cited by title and section):
+
+* [P3] "从Attention矩阵到显存读写：FlashAttention真正解决的痛点" (lab write-up,
+  dpshk.com): §2.1 the three-step definition S = Q K^T, P = softmax(S) along
+  the last dimension, O = P V; §3.2 the online-softmax recurrence with running
+  row max m and exp-sum l; §3.3 recomputation in the backward pass; §4.2 the
+  [batch, seqlen, heads, head_dim] layout, ``softmax_scale`` (default 1/sqrt(d))
+  and ``causal``.
+* [P4] "使用FlashAttention优化PyTorch模型注意力计算" (tiemojia.cn), section
+  "FlashAttention 是如何做到又快又省内存的": the einsum form of standard
+  attention, scores divided by sqrt(d_head), softmax over the key axis.
+
+The method is mathematically the plain definition ([P3] §3.2 states the tiled
+form is equivalent to the global softmax; [P4] calls it "数学上等价"), so the
+forward oracle *is* that definition, materialising S and P in full for each
+(batch, head). The pages give no backward formulas; the backward oracle is the
+textbook chain rule through the softmax Jacobian (the plain reading):
+
+    dV = P^T dO;  dP = dO V^T;  D_i = sum_j P_ij dP_ij;  dS = P o (dP - D)
+    dQ = scale * dS K;  dK = scale * dS^T Q
+
+``online_softmax_forward`` restates the tiled recurrence of [P3] §3.2 step by
+step (in fp64); it is pinned against the direct definition in the tests.
+
+Masking reading: ``causal`` keeps key j for query i iff j <= i (queries and keys
+have the same length, so the mask is aligned top-left). Row logsumexp (LSE) is
+the natural log of sum_j exp(scale * q_i . k_j) over kept keys; the pages do not
+define it, it is what the backward recompute needs.
+
+Every function here is pinned by a test in ``tests/test_oracle_pins.py`` to
+something other than itself (closed forms, invariants, brute force, a hand-worked
+example, central finite differences).
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+ROW_BLOCK = 512  # rows of S materialised at once for long sequences
+
+
+def _as_f64(x) -> np.ndarray:
+    a = np.asarray(x, dtype=np.float64)
+    if a.ndim != 4:
+        raise ValueError("expected a [batch, seqlen, heads, head_dim] array")
+    return a
+
+
+def _scores(qh: np.ndarray, kh: np.ndarray, scale: float, rows: np.ndarray, causal: bool) -> np.ndarray:
+    """S = scale * Q K^T for the given query rows of one head ([P3] §2.1 step 1).
+
+    Causal: entries with key index j > query index i are -inf (excluded).
+    """
+    s = scale * (qh[rows] @ kh.T)
+    if causal:
+        keys = np.arange(kh.shape[0])
+        s[keys[None, :] > rows[:, None]] = -np.inf
+    return s
+
+
+def _softmax_rows(s: np.ndarray):
+    """P = softmax(S) along the key axis ([P3] §2.1 step 2), and the row LSE."""
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    l = e.sum(axis=1, keepdims=True)
+    return e / l, (m + np.log(l))[:, 0]
+
+
+def attention_forward(q, k, v, scale: float, causal: bool = False, rows=None):
+    """O = softmax(scale Q K^T [+causal mask]) V and LSE, in fp64.
+
+    q, k, v: [B, N, H, d]. Returns (O [B, N, H, d], LSE [B, H, N]).
+    ``rows``: optional 1-D array of query rows to evaluate (each row is
+    independent); the other rows of O / LSE are NaN.
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, N, H, d = q.shape
+    if k.shape != (B, N, H, d) or v.shape != (B, N, H, d):
+        raise ValueError("q, k, v must share the shape [B, N, H, d]")
+    all_rows = np.arange(N) if rows is None else np.asarray(rows, dtype=np.int64)
+    o = np.full((B, N, H, d), np.nan)
+    lse = np.full((B, H, N), np.nan)
+    for b in range(B):
+        for h in range(H):
+            qh, kh, vh = q[b, :, h, :], k[b, :, h, :], v[b, :, h, :]
+            for r0 in range(0, len(all_rows), ROW_BLOCK):
+                rr = all_rows[r0:r0 + ROW_BLOCK]
+                p, lse_rows = _softmax_rows(_scores(qh, kh, scale, rr, causal))
+                o[b, rr, h, :] = p @ vh          # [P3] §2.1 step 3
+                lse[b, h, rr] = lse_rows
+    return o, lse
+
+
+def attention_backward(q, k, v, do, scale: float, causal: bool = False, heads=None):
+    """Gradients (dQ, dK, dV) of L = sum(dO o O) for the attention above, fp64.
+
+    ``heads``: optional list of (b, h) pairs to evaluate (dK/dV of a head need
+    every query row, so sampling is per head); other heads are NaN.
+    Also returns D [B, H, N] = rowsum(P o dP), which equals rowsum(dO o O).
+    """
+    q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
+    B, N, H, d = q.shape
+    dq = np.full_like(q, np.nan)
+    dk = np.full_like(q, np.nan)
+    dv = np.full_like(q, np.nan)
+    dd = np.full((B, H, N), np.nan)
+    pairs = [(b, h) for b in range(B) for h in range(H)] if heads is None else list(heads)
+    rows = np.arange(N)
+    for b, h in pairs:
+        qh, kh, vh, doh = q[b, :, h, :], k[b, :, h, :], v[b, :, h, :], do[b, :, h, :]
+        p, _ = _softmax_rows(_scores(qh, kh, scale, rows, causal))
+        dvh = p.T @ doh
+        dp = doh @ vh.T
+        drow = (p * dp).sum(axis=1)
+        ds = p * (dp - drow[:, None])
+        dq[b, :, h, :] = scale * (ds @ kh)
+        dk[b, :, h, :] = scale * (ds.T @ qh)
+        dv[b, :, h, :] = dvh
+        dd[b, h, :] = drow
+    return dq, dk, dv, dd
+
+
+def online_softmax_forward(q, k, v, scale: float, causal: bool, tile_sizes):
+    """The tiled online-softmax forward of [P3] §3.2, one key tile at a time.
+
+    For each query row, keep the running max m and exp-sum l; for each key tile
+    j with local scores s: m_new = max(m, max(s)); O <- O * e^(m - m_new) +
+    e^(s - m_new) V_j; l <- l * e^(m - m_new) + sum e^(s - m_new); at the end
+    O <- O / l. ``tile_sizes`` lists the widths of the consecutive key tiles
+    (they must add up to N). Returns (O, LSE) with LSE = m + ln l.
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, N, H, d = q.shape
+    if sum(tile_sizes) != N:
+        raise ValueError("tile sizes must cover the key axis exactly")
+    o = np.empty((B, N, H, d))
+    lse = np.empty((B, H, N))
+    rows = np.arange(N)
+    for b in range(B):
+        for h in range(H):
+            qh, kh, vh = q[b, :, h, :], k[b, :, h, :], v[b, :, h, :]
+            m = np.full(N, -np.inf)
+            l = np.zeros(N)
+            acc = np.zeros((N, d))
+            start = 0
+            for width in tile_sizes:
+                cols = np.arange(start, start + width)
+                s = scale * (qh @ kh[cols].T)
+                if causal:
+                    s[cols[None, :] > rows[:, None]] = -np.inf
+                m_new = np.maximum(m, s.max(axis=1))
+                # rows with nothing kept so far keep m = -inf; guard their factors
+                alive = np.isfinite(m_new)
+                alpha = np.where(alive, np.exp(np.where(alive, m - m_new, 0.0)), 1.0)
+                e = np.where(alive[:, None], np.exp(s - np.where(alive, m_new, 0.0)[:, None]), 0.0)
+                acc = acc * alpha[:, None] + e @ vh[cols]
+                l = l * alpha + e.sum(axis=1)
+                m = m_new
+                start += width
+            o[b, :, h, :] = acc / l[:, None]
+            lse[b, h, :] = m + np.log(l)
+    return o, lse
+
+
+def default_scale(d: int) -> float:
+    """softmax_scale=None means 1/sqrt(head_dim) ([P3] §4.2 and §6.2)."""
+    return 1.0 / math.sqrt(d)

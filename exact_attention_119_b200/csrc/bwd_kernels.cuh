@@ -1,0 +1,676 @@
+// Backward kernels: dQ, dK, dV of O = softmax(scale Q K^T [+causal]) V.
+//
+// The lab write-up "从Attention矩阵到显存读写：FlashAttention真正解决的痛点"
+// (§3.3) recomputes S and P in the backward pass instead of storing them; the
+// pages give no gradient formulas, so these kernels implement the chain rule
+// through softmax, with P rebuilt from the forward's row LSE:
+//
+//   P = exp(scale S - LSE),  dV = P^T dO,  dP = dO V^T,
+//   D_i = rowsum(dO o O)_i,  dS = P o (dP - D),  dK = scale dS^T Q,
+//   dQ = scale dS K.
+//
+// Three launches on the caller's stream:
+//   1. fa_bwd_prep:  D and LSE*log2(e) into padded per-head arrays; zeroes the
+//                    dQ ordering counters and the work counter.
+//   2. fa_bwd_dkdv:  persistent; one CTA per SM fetches work items (b, h, key
+//                    tile j) in increasing order. Per item K_j, V_j stay in
+//                    shared memory and dK_j, dV_j accumulate in TMEM while
+//                    (Q_i, dO_i) tiles stream through a 2-stage ring for
+//                    i = last .. first (descending). Per step, five tcgen05
+//                    MMAs: S^T = K Q^T, dP^T = V dO^T, dV += P^T dO,
+//                    dQ_part = dS K, dK += dS^T Q. dQ_part is added into an
+//                    fp32 accumulator in ascending j order (a per-tile
+//                    counter says whose turn it is), so the sum is
+//                    deterministic.
+//   3. fa_bwd_dq:    dQ = scale * accumulator, cast to fp16/bf16.
+//
+// Ordering cannot deadlock: items start in increasing index order (a global
+// atomic counter), an item only waits for the item of key tile j-1 of the
+// same head, which has a lower index and so has already started; the lowest
+// unfinished item never waits. Every wait is bounded anyway.
+#pragma once
+
+#include <algorithm>
+
+#include "sm100.cuh"
+
+namespace fa {
+
+// Workspace layout (all offsets 256-byte aligned).
+struct BwdLayout {
+  int npad, ntiles;
+  size_t off_lse2, off_dd, off_dqacc, off_cnt, off_sched;
+  size_t total_bytes;
+  static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+  static BwdLayout make(int B, int N, int H, int d) {
+    BwdLayout L;
+    L.ntiles = (N + 127) / 128;
+    L.npad = L.ntiles * 128;
+    const size_t bh = (size_t)B * H;
+    size_t off = 0;
+    L.off_lse2 = off;  off = up256(off + bh * L.npad * 4);
+    L.off_dd = off;    off = up256(off + bh * L.npad * 4);
+    L.off_dqacc = off; off = up256(off + bh * L.npad * (size_t)d * 4);
+    L.off_cnt = off;   off = up256(off + bh * L.ntiles * 4);
+    L.off_sched = off; off = up256(off + 16);
+    L.total_bytes = off;
+    return L;
+  }
+};
+
+struct BwdArgs {
+  const uint16_t* o;
+  const uint16_t* dout;
+  const float* lse;
+  uint16_t* dq;
+  uint16_t* dk;
+  uint16_t* dv;
+  float* lse2;   // [B*H, npad] LSE * log2(e); +inf on pad rows
+  float* dd;     // [B*H, npad] D; 0 on pad rows
+  float* dqacc;  // [B*H, ntiles, d/4, 128, 4] fp32
+  int* cnt;      // [B*H, ntiles] dQ ordering counters
+  int* sched;    // work counter
+  int B, N, H, npad, ntiles;
+  float scale;       // softmax_scale
+  float scale_log2;  // softmax_scale * log2(e)
+};
+
+// ------------------------------------------------------------------ kernel 1
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_prep(const BwdArgs a) {
+  // A group of G = D/8 lanes per (b, n, h) row, 8 elements per lane; the
+  // warp's groups take consecutive rows so the loop stays warp-uniform.
+  constexpr int G = D / 8;
+  const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const long long nthreads = (long long)gridDim.x * blockDim.x;
+  const long long rows = (long long)a.B * a.N * a.H;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane % G;
+  const long long ngroups = nthreads / G;
+  for (long long row0 = (tid / 32) * (32 / G); row0 < rows; row0 += ngroups) {
+    const long long row = row0 + lane / G;
+    const bool valid = row < rows;
+    float acc = 0.f;
+    if (valid) {
+      const uint4 ov = reinterpret_cast<const uint4*>(a.o + row * D)[sub];
+      const uint4 dv = reinterpret_cast<const uint4*>(a.dout + row * D)[sub];
+      const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
+      const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 x = unpack2<BF16>(ow[i]);
+        const float2 y = unpack2<BF16>(dw[i]);
+        acc = fmaf(x.x, y.x, acc);
+        acc = fmaf(x.y, y.y, acc);
+      }
+    }
+#pragma unroll
+    for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, G);
+    if (valid && sub == 0) {
+      const int h = (int)(row % a.H);
+      const long long bn = row / a.H;
+      const int n = (int)(bn % a.N);
+      const int b = (int)(bn / a.N);
+      const size_t idx = ((size_t)b * a.H + h) * a.npad + n;
+      a.dd[idx] = acc;
+      a.lse2[idx] = a.lse[((size_t)b * a.H + h) * a.N + n] * 1.4426950408889634f;
+    }
+  }
+  // Pad rows (no query there: P = 0 through LSE = +inf), counters, work counter.
+  const int padn = a.npad - a.N;
+  const long long pads = (long long)a.B * a.H * padn;
+  for (long long p = tid; p < pads; p += nthreads) {
+    const long long bh = p / padn;
+    const int n = a.N + (int)(p % padn);
+    a.dd[bh * a.npad + n] = 0.f;
+    a.lse2[bh * a.npad + n] = INFINITY;
+  }
+  const long long ncnt = (long long)a.B * a.H * a.ntiles;
+  for (long long p = tid; p < ncnt; p += nthreads) a.cnt[p] = 0;
+  if (tid == 0) *a.sched = 0;
+}
+
+// ------------------------------------------------------------------ kernel 3
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_dq(const BwdArgs a) {
+  // Thread per (row, 4 columns); consecutive threads take consecutive rows of
+  // one tile so the accumulator reads are contiguous.
+  const long long total = (long long)a.B * a.H * a.npad * (D / 4);
+  for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < total;
+       t += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(t % 128);
+    long long rest = t / 128;
+    const int c4 = (int)(rest % (D / 4));
+    rest /= (D / 4);
+    const int tile = (int)(rest % a.ntiles);
+    const long long bh = rest / a.ntiles;
+    const int n = tile * 128 + r;
+    if (n >= a.N) continue;
+    const float4 v = reinterpret_cast<const float4*>(a.dqacc)[t];
+    const int b = (int)(bh / a.H), h = (int)(bh % a.H);
+    uint16_t* dst = a.dq + (((size_t)b * a.N + n) * a.H + h) * D + c4 * 4;
+    uint2 w;
+    w.x = pack2<BF16>(v.x * a.scale, v.y * a.scale);
+    w.y = pack2<BF16>(v.z * a.scale, v.w * a.scale);
+    *reinterpret_cast<uint2*>(dst) = w;
+  }
+}
+
+// ------------------------------------------------------------------ kernel 2
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kTile = 128 * D * 2;  // one 128-row tile of Q/K/V/dO
+  static constexpr int kBox = 128 * 128;     // one 64-column box of a tile
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kTile;
+  static constexpr int kQ = kV + kTile;            // 2 stages
+  static constexpr int kDO = kQ + 2 * kTile;       // 2 stages
+  static constexpr int kDS = kDO + 2 * kTile;      // dS^T, 128 x 128 16-bit
+  static constexpr int kLSE = kDS + 128 * 128 * 2; // 2 stages x 128 fp32
+  static constexpr int kDD = kLSE + 2 * 512;       // 2 stages x 128 fp32
+  static constexpr int kBar = kDD + 2 * 512;
+  static constexpr int kSmem = kBar + 384;
+  // TMEM columns
+  static constexpr uint32_t kTdV = 0;
+  static constexpr uint32_t kTdK = D;
+  static constexpr uint32_t kTS = 2 * D;        // S^T, then P^T (16-bit) in place
+  static constexpr uint32_t kTdP = 2 * D + 128; // dP^T, then the dQ partial
+  static constexpr int kThreads = 512;
+};
+
+struct BwdBarriers {
+  uint64_t kv_full, kv_empty;
+  uint64_t qdo_full[2], qdo_empty[2];
+  uint64_t s_full, dp_full, p_ready, ds_ready, ds_free, dq_full, dq_empty;
+  uint64_t acc_full, acc_empty, drain;
+  uint64_t item_full[2], item_empty[2];
+  uint64_t dq_turn, dq_added;  // dQ warpgroup: "our turn to add", "all added"
+  int item[2];
+  int dq_go;     // the ordering wait succeeded
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+
+// Work item -> (bh, j) and the q-tile range [i_lo, ntiles).
+struct BwdItem {
+  int bh, j, i_lo, T;
+};
+__device__ __forceinline__ BwdItem decode_item(int item, int ntiles, bool causal) {
+  BwdItem it;
+  it.bh = item / ntiles;
+  it.j = item % ntiles;
+  it.i_lo = causal ? it.j : 0;
+  it.T = ntiles - it.i_lo;
+  return it;
+}
+
+template <int D, bool CAUSAL, bool BF16>
+__global__ void __launch_bounds__(512, 1)
+    fa_bwd_dkdv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const BwdArgs a) {
+  using C = BwdCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (smem_u32(smem) & 1023u) {  // the swizzled tiles need a 1 KB aligned base
+    if (threadIdx.x == 0) atomicCAS(&g_status, 0, 3 /*FA_ERR_CUDA*/);
+    return;
+  }
+  BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + C::kBar);
+  volatile int* abort = &bars->abort;
+  const int total_items = a.B * a.H * a.ntiles;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->kv_full, 1);
+    mbar_init(&bars->kv_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->qdo_full[s], 1);
+      mbar_init(&bars->qdo_empty[s], 1);
+      mbar_init(&bars->item_full[s], 1);
+      mbar_init(&bars->item_empty[s], 13);  // MMA thread + 8 compute warps + 4 dQ warps
+    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->dp_full, 1);
+    mbar_init(&bars->p_ready, 256);
+    mbar_init(&bars->ds_ready, 256);
+    mbar_init(&bars->ds_free, 1);
+    mbar_init(&bars->dq_full, 1);
+    mbar_init(&bars->dq_empty, 128);
+    mbar_init(&bars->acc_full, 1);
+    mbar_init(&bars->acc_empty, 256);
+    mbar_init(&bars->drain, 1);
+    mbar_init(&bars->dq_turn, 1);
+    mbar_init(&bars->dq_added, 128);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 12) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  // Register split per SM sub-partition (one warp of each warpgroup on each):
+  // producer/MMA 112 + compute 120 + compute 120 + dQ 160 = 512 = the 4 x 128
+  // the CTA was launched with, so the one setmaxnreg.inc cannot wait forever.
+  if (warp >= 12) {
+    reg_alloc_dec<112>();
+    if (warp == 12 && elect_one()) {
+      // ------------------------------------------------------------ producer
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      int g = 0;          // Q/dO loads issued (global step counter)
+      int n_item = 0;     // items taken by this CTA
+      int kv_loads = 0;   // K/V loads issued
+      bool ok = true;
+      while (ok) {
+        const int slot = n_item & 1;
+        if (n_item >= 2) ok = mbar_wait(&bars->item_empty[slot], ((n_item >> 1) & 1) ^ 1, abort);
+        if (!ok) break;
+        const int item = atomicAdd(a.sched, 1);
+        bars->item[slot] = item < total_items ? item : -1;
+        mbar_arrive(&bars->item_full[slot]);
+        if (item >= total_items) break;
+        const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
+        const int b = w.bh / a.H, h = w.bh % a.H;
+        for (int k = 0; k < w.T && ok; ++k) {
+          const int st = g & 1;
+          const int i = a.ntiles - 1 - k;
+          if (g >= 2) ok = mbar_wait(&bars->qdo_empty[st], ((g >> 1) & 1) ^ 1, abort);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bars->qdo_full[st], 2 * C::kTile + 1024);
+          for (int kb = 0; kb < D / 64; ++kb) {
+            tma_load_4d(&tm_q, smem + C::kQ + st * C::kTile + kb * C::kBox, &bars->qdo_full[st], kb * 64, h,
+                        i * 128, b);
+            tma_load_4d(&tm_do, smem + C::kDO + st * C::kTile + kb * C::kBox, &bars->qdo_full[st], kb * 64, h,
+                        i * 128, b);
+          }
+          bulk_load(smem + C::kLSE + st * 512, a.lse2 + (size_t)w.bh * a.npad + i * 128, 512, &bars->qdo_full[st]);
+          bulk_load(smem + C::kDD + st * 512, a.dd + (size_t)w.bh * a.npad + i * 128, 512, &bars->qdo_full[st]);
+          ++g;
+          if (k == 0) {
+            // K_j, V_j once the previous item released them (after this
+            // item's first Q/dO load is already on its way).
+            if (kv_loads >= 1) ok = mbar_wait(&bars->kv_empty, (kv_loads - 1) & 1, abort);
+            if (!ok) break;
+            mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTile);
+            for (int kb = 0; kb < D / 64; ++kb) {
+              tma_load_4d(&tm_k, smem + C::kK + kb * C::kBox, &bars->kv_full, kb * 64, h, w.j * 128, b);
+              tma_load_4d(&tm_v, smem + C::kV + kb * C::kBox, &bars->kv_full, kb * 64, h, w.j * 128, b);
+            }
+            ++kv_loads;
+          }
+        }
+        ++n_item;
+      }
+      // Never leave with copies in flight: the last load of each stage, and
+      // the last K/V load.
+      for (int x = (g > 2 ? g - 2 : 0); x < g; ++x) mbar_wait(&bars->qdo_full[x & 1], (x >> 1) & 1, abort, false);
+      if (kv_loads >= 1) mbar_wait(&bars->kv_full, (kv_loads - 1) & 1, abort, false);
+    } else if (warp == 13 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr uint32_t kIdSq = idesc_f16(BF16, 128, 128, false, false);  // S^T, dP^T
+      constexpr uint32_t kIdKM = idesc_f16(BF16, 128, D, false, true);     // dV (A in TMEM), dK
+      constexpr uint32_t kIdQ = idesc_f16(BF16, 128, D, true, true);       // dQ part: A = dS (MN-major)
+      // Descriptors of the tile bases; a K step only moves the start-address
+      // field (bits 0-13, in 16-byte units), which cannot carry out of it here.
+      const uint64_t dK_k = sdesc(smem_u32(smem + C::kK), 16, 1024);
+      const uint64_t dV_k = sdesc(smem_u32(smem + C::kV), 16, 1024);
+      const uint64_t dQ_k = sdesc(smem_u32(smem + C::kQ), 16, 1024);
+      const uint64_t dDO_k = sdesc(smem_u32(smem + C::kDO), 16, 1024);
+      const uint64_t dDS_k = sdesc(smem_u32(smem + C::kDS), 16, 1024);
+      const uint64_t dK_mn = sdesc(smem_u32(smem + C::kK), C::kBox, 1024);
+      const uint64_t dQ_mn = sdesc(smem_u32(smem + C::kQ), C::kBox, 1024);
+      const uint64_t dDO_mn = sdesc(smem_u32(smem + C::kDO), C::kBox, 1024);
+      const uint64_t dDS_mn = sdesc(smem_u32(smem + C::kDS), C::kBox, 1024);
+      constexpr uint32_t kStage16 = C::kTile >> 4;
+      auto kstep = [](int ks) { return (uint64_t)(((ks / 4) * C::kBox + (ks % 4) * 32) >> 4); };
+      auto mstep = [](int kk) { return (uint64_t)((kk * 2048) >> 4); };
+      auto issue_st = [&](uint64_t a0, uint64_t b0, uint32_t dst) {  // [128 x 128] over d
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) mma_ss(tmem + dst, a0 + kstep(ks), b0 + kstep(ks), kIdSq, ks > 0);
+      };
+      int g = 0, n_item = 0;
+      bool ok = true;
+      while (ok) {
+        const int slot = n_item & 1;
+        ok = mbar_wait(&bars->item_full[slot], (n_item >> 1) & 1, abort);
+        if (!ok) break;
+        const int item = bars->item[slot];
+        mbar_arrive(&bars->item_empty[slot]);
+        if (item < 0) break;
+        const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
+        ok = mbar_wait(&bars->kv_full, n_item & 1, abort) && mbar_wait(&bars->qdo_full[g & 1], (g >> 1) & 1, abort);
+        if (!ok) break;
+        tc_fence_after();
+        issue_st(dK_k, dQ_k + (g & 1) * kStage16, C::kTS);
+        mma_commit(&bars->s_full);
+        if (g > 0) ok = mbar_wait(&bars->dq_empty, (g - 1) & 1, abort);
+        if (!ok) break;
+        tc_fence_after();
+        issue_st(dV_k, dDO_k + (g & 1) * kStage16, C::kTdP);
+        mma_commit(&bars->dp_full);
+        for (int k = 0; k < w.T && ok; ++k, ++g) {
+          const int st = g & 1;
+          ok = mbar_wait(&bars->p_ready, g & 1, abort);
+          if (ok && k == 0 && n_item > 0) ok = mbar_wait(&bars->acc_empty, (n_item - 1) & 1, abort);
+          if (!ok) break;
+          tc_fence_after();
+          // dV += P^T dO   (A = P^T in TMEM, 16-bit packed)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + C::kTdV, tmem + C::kTS + kk * 8 + (kk >= 4 ? 32 : 0), dDO_mn + st * kStage16 + mstep(kk),
+                   kIdKM, (k > 0 || kk > 0));
+          if (k + 1 < w.T) {
+            ok = mbar_wait(&bars->qdo_full[(g + 1) & 1], ((g + 1) >> 1) & 1, abort);
+            if (!ok) break;
+            issue_st(dK_k, dQ_k + ((g + 1) & 1) * kStage16, C::kTS);
+            mma_commit(&bars->s_full);
+          }
+          ok = mbar_wait(&bars->ds_ready, g & 1, abort);
+          if (!ok) break;
+          tc_fence_after();
+          // dQ_part = dS K   (A = dS: dS^T stored [key][query] -> MN-major)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) mma_ss(tmem + C::kTdP, dDS_mn + mstep(kk), dK_mn + mstep(kk), kIdQ, kk > 0);
+          mma_commit(&bars->dq_full);
+          // dK += dS^T Q   (A = dS^T K-major)
+#pragma unroll
+          for (int kq = 0; kq < 8; ++kq)
+            mma_ss(tmem + C::kTdK, dDS_k + kstep(kq), dQ_mn + st * kStage16 + mstep(kq), kIdKM, (k > 0 || kq > 0));
+          mma_commit(&bars->ds_free);
+          mma_commit(&bars->qdo_empty[st]);
+          if (k + 1 < w.T) {
+            ok = mbar_wait(&bars->dq_empty, g & 1, abort);
+            if (!ok) break;
+            tc_fence_after();
+            issue_st(dV_k, dDO_k + ((g + 1) & 1) * kStage16, C::kTdP);
+            mma_commit(&bars->dp_full);
+          }
+        }
+        if (!ok) break;
+        mma_commit(&bars->acc_full);
+        mma_commit(&bars->kv_empty);
+        ++n_item;
+      }
+      mma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0, abort, false);
+    }
+  } else if (warp < 8) {
+    reg_alloc_dec<120>();
+    // ------------------------------------------------------- compute warps
+    // Thread = key row c (TMEM lane); warpgroup wg takes query columns
+    // [64 wg, 64 wg + 64) of each 128 x 128 step.
+    const int wg = warp / 4;
+    const int quad = warp % 4;
+    const int c = quad * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const float cl2 = a.scale_log2;
+    const float* sLSE = reinterpret_cast<const float*>(smem + C::kLSE);
+    const float* sDD = reinterpret_cast<const float*>(smem + C::kDD);
+    uint8_t* sDS = smem + C::kDS + wg * C::kBox;  // this warpgroup's 64 query columns
+    int g = 0, n_item = 0;
+    bool ok = true;
+    while (ok) {
+      const int slot = n_item & 1;
+      ok = mbar_wait_warp(&bars->item_full[slot], (n_item >> 1) & 1, abort);
+      if (!ok) break;
+      const int item = bars->item[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->item_empty[slot]);
+      if (item < 0) break;
+      const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
+      const int key = w.j * 128 + c;
+      for (int k = 0; k < w.T; ++k, ++g) {
+        const int st = g & 1;
+        const int i = a.ntiles - 1 - k;
+        const bool diag = CAUSAL && i == w.j;
+        // ---- P^T = exp2(S^T * c - LSE2) for this thread's 64 queries
+        if (!mbar_wait_warp(&bars->s_full, g & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        // P^T of queries [64 wg, 64 wg + 64), packed two per 32-bit word.
+        uint32_t pk[32];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t s[32];
+          tmem_ld32(lane_base + C::kTS + wg * 64 + h2 * 32, s);
+          tmem_ld_wait();
+          tie_regs32(s);
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const int qc = wg * 64 + h2 * 32 + 2 * x;
+            float v0 = ex2(fmaf(__uint_as_float(s[2 * x]), cl2, -sLSE[st * 128 + qc]));
+            float v1 = ex2(fmaf(__uint_as_float(s[2 * x + 1]), cl2, -sLSE[st * 128 + qc + 1]));
+            if (diag && key > i * 128 + qc) v0 = 0.f;
+            if (diag && key > i * 128 + qc + 1) v1 = 0.f;
+            pk[h2 * 16 + x] = pack2<BF16>(v0, v1);
+          }
+        }
+        // It goes into columns [64 wg, 64 wg + 32) of S: columns this
+        // warpgroup has already read, so the other warpgroup's S is untouched.
+        tmem_st32(lane_base + C::kTS + wg * 64, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars->p_ready);
+        // ---- dS^T = P^T o (dP^T - D) -> shared memory (16-bit), from the same
+        // rounded P that the dV product uses.
+        if (!mbar_wait_warp(&bars->dp_full, g & 1, abort)) { ok = false; break; }
+        if (g > 0 && !mbar_wait_warp(&bars->ds_free, (g - 1) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t dp[32];
+          tmem_ld32(lane_base + C::kTdP + wg * 64 + h2 * 32, dp);
+          tmem_ld_wait();
+          tie_regs32(dp);
+          uint32_t dsk[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const int qc = wg * 64 + h2 * 32 + 2 * x;
+            const float2 pp = unpack2<BF16>(pk[h2 * 16 + x]);
+            const float d0 = pp.x * (__uint_as_float(dp[2 * x]) - sDD[st * 128 + qc]);
+            const float d1 = pp.y * (__uint_as_float(dp[2 * x + 1]) - sDD[st * 128 + qc + 1]);
+            dsk[x] = pack2<BF16>(d0, d1);
+          }
+          // Row c of a 128-byte-swizzled [128][64] box: 16-byte chunk x goes
+          // to x ^ (c % 8).
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const int chunk = h2 * 4 + x;
+            uint4* dst = reinterpret_cast<uint4*>(sDS + c * 128 + ((chunk ^ (c & 7)) * 16));
+            *dst = make_uint4(dsk[4 * x], dsk[4 * x + 1], dsk[4 * x + 2], dsk[4 * x + 3]);
+          }
+        }
+        tc_fence_before();  // dP^T reads done before the dQ MMA reuses these columns
+        fence_proxy_async_smem();
+        mbar_arrive(&bars->ds_ready);
+      }
+      if (!ok) break;
+      // ---- epilogue: warpgroup 0 stores dV_j, warpgroup 1 stores scale * dK_j
+      if (!mbar_wait_warp(&bars->acc_full, n_item & 1, abort)) { ok = false; break; }
+      tc_fence_after();
+      {
+        const int b = w.bh / a.H, h = w.bh % a.H;
+        const bool valid = key < a.N;
+        const float mul = wg == 0 ? 1.f : a.scale;
+        uint16_t* dst = (wg == 0 ? a.dv : a.dk) + (((size_t)b * a.N + (valid ? key : 0)) * a.H + h) * D;
+        const uint32_t src = lane_base + (wg == 0 ? C::kTdV : C::kTdK);
+#pragma unroll 1
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t v[32];
+          tmem_ld32(src + q * 32, v);
+          tmem_ld_wait();
+          tie_regs32(v);
+          uint32_t pk[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            pk[x] = pack2<BF16>(__uint_as_float(v[2 * x]) * mul, __uint_as_float(v[2 * x + 1]) * mul);
+          if (valid) {
+            uint4* o4 = reinterpret_cast<uint4*>(dst + q * 32);
+#pragma unroll
+            for (int y = 0; y < 4; ++y) o4[y] = make_uint4(pk[4 * y], pk[4 * y + 1], pk[4 * y + 2], pk[4 * y + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->acc_empty);
+      ++n_item;
+    }
+  } else {
+    reg_alloc_inc<160>();
+    // ------------------------------------------------------ dQ warps (8-11)
+    // Thread = query row r of the step (TMEM lane).
+    const int quad = warp % 4;
+    const int r = quad * 32 + lane;
+    const uint32_t src = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::kTdP;
+    int g = 0, n_item = 0;
+    bool ok = true;
+    while (ok) {
+      const int slot = n_item & 1;
+      ok = mbar_wait_warp(&bars->item_full[slot], (n_item >> 1) & 1, abort);
+      if (!ok) break;
+      const int item = bars->item[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->item_empty[slot]);
+      if (item < 0) break;
+      const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
+      for (int k = 0; k < w.T; ++k, ++g) {
+        const int i = a.ntiles - 1 - k;
+        // The warpgroup synchronises through two mbarriers (bounded waits, no
+        // named barriers), so a warp that gives up cannot strand the others.
+        const bool got = mbar_wait_warp(&bars->dq_full, g & 1, abort);
+        uint32_t v[D];
+        if (got) {
+          tc_fence_after();
+#pragma unroll
+          for (int q = 0; q < D / 32; ++q) tmem_ld32(src + q * 32, v + q * 32);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < D / 32; ++q) tie_regs32(v + q * 32);
+          tc_fence_before();
+          mbar_arrive(&bars->dq_empty);
+        }
+        // Thread 256 waits until key tile j-1 of this head has added its part
+        // of tile i, then opens the turn for the warpgroup.
+        const size_t tile = (size_t)w.bh * a.ntiles + i;
+        int* cnt = a.cnt + tile;
+        if (threadIdx.x == 256) {
+          bool go = got;
+          if (go && w.j > 0 && ld_acquire(cnt) != w.j) {
+            const uint64_t t0 = globaltimer();
+            for (uint32_t n = 1;; ++n) {
+              if (ld_acquire(cnt) == w.j) break;
+              if ((n & 63u) == 0) {
+                if (*abort) { go = false; break; }
+                if (globaltimer() - t0 > FA_WAIT_LIMIT_NS) {
+                  record_timeout(2);
+                  *abort = 1;
+                  go = false;
+                  break;
+                }
+              }
+              __nanosleep(64);
+            }
+          }
+          bars->dq_go = go ? 1 : 0;
+          mbar_arrive(&bars->dq_turn);
+        }
+        const bool turn = mbar_wait(&bars->dq_turn, g & 1, abort) && bars->dq_go;
+        const bool step_ok = got && turn;
+        if (step_ok) {
+          float* acc = a.dqacc + tile * 128 * D;
+#pragma unroll
+          for (int q = 0; q < D / 4; ++q) {
+            float* p4 = acc + ((size_t)q * 128 + r) * 4;
+            if (w.j == 0)
+              *reinterpret_cast<float4*>(p4) = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                                           __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+            else
+              red_add_v4(p4, __uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
+                         __uint_as_float(v[4 * q + 3]));
+          }
+          __threadfence();
+        }
+        mbar_arrive(&bars->dq_added);
+        if (threadIdx.x == 256) {
+          // Publish only when all 128 rows are in; otherwise the next key
+          // tile's wait runs out and reports the timeout.
+          if (mbar_wait(&bars->dq_added, g & 1, abort) && step_ok) st_release(cnt, w.j + 1);
+        }
+        if (!step_ok) { ok = false; break; }
+      }
+      if (!ok) break;
+      ++n_item;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 12) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------- launch
+
+template <int D, bool CAUSAL, bool BF16>
+cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const CUtensorMap& mdo, const BwdArgs& a, int num_sms, cudaStream_t s) {
+  using C = BwdCfg<D>;
+  const long long rows = (long long)a.B * a.N * a.H;
+  const int prep_blocks = (int)std::min<long long>((rows * (D / 8) + 255) / 256 + 1, 4LL * num_sms * 8);
+  fa_bwd_prep<D, BF16><<<prep_blocks, 256, 0, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  auto kern = fa_bwd_dkdv<D, CAUSAL, BF16>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  const int items = a.B * a.H * a.ntiles;
+  const int grid = std::min(items, num_sms);
+  kern<<<grid, C::kThreads, C::kSmem, s>>>(mq, mk, mv, mdo, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long dq_threads = (long long)a.B * a.H * a.npad * (D / 4);
+  const int dq_blocks = (int)std::min<long long>((dq_threads + 255) / 256, 64LL * num_sms);
+  fa_bwd_dq<D, BF16><<<dq_blocks, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace fa

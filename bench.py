@@ -130,6 +130,22 @@ def dist_env():
     return world, rank, local
 
 
+def reduce_max(values, world, device=None):
+    """Element-wise max over ranks of a list of floats (identity when world == 1)."""
+    if world == 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_tflops(world, steps, flops_per_step, max_ms):
+    """Throughput of the whole job: every rank's FLOPs over the slowest rank's time."""
+    return world * steps * flops_per_step / (max_ms * 1e-3) / 1e12
+
+
 def oracle_sample(workload, budget_s=15.0, max_heads=None):
     """Time the fp64 oracle on whole heads of the workload until budget_s."""
     import numpy as np
@@ -265,15 +281,12 @@ def main():
     fwd_ms = [e[0].elapsed_time(e[1]) for e in ev]
     bwd_ms = [e[1].elapsed_time(e[2]) for e in ev]
     tot_ms = sum(fwd_ms) + sum(bwd_ms)
-    t = torch.tensor([tot_ms, sum(fwd_ms), sum(bwd_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    tot_ms, fwd_sum, bwd_sum = t.tolist()
+    tot_ms, fwd_sum, bwd_sum = reduce_max([tot_ms, sum(fwd_ms), sum(bwd_ms)], world, dev)
 
     f_fwd, f_bwd = flops(B, N, H, d, causal)
-    value = world * args.steps * (f_fwd + f_bwd) / (tot_ms * 1e-3) / 1e12
-    fwd_tflops = world * args.steps * f_fwd / (fwd_sum * 1e-3) / 1e12
-    bwd_tflops = world * args.steps * f_bwd / (bwd_sum * 1e-3) / 1e12
+    value = whole_job_tflops(world, args.steps, f_fwd + f_bwd, tot_ms)
+    fwd_tflops = whole_job_tflops(world, args.steps, f_fwd, fwd_sum)
+    bwd_tflops = whole_job_tflops(world, args.steps, f_bwd, bwd_sum)
 
     # ---- end to end through the public API: pinned host in, results back out
     out_host = {n: torch.empty_like(host["q"]).pin_memory() for n in ("o", "dq", "dk", "dv")}
@@ -295,11 +308,10 @@ def main():
         out_host["dv"].copy_(dv, non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in e2e_ev)], dtype=torch.float64, device=dev)
+    (e2e_ms,) = reduce_max([sum(a.elapsed_time(b) for a, b in e2e_ev)], world, dev)
     if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
         dist.barrier()
-    e2e_value = world * args.steps * (f_fwd + f_bwd) / (e2e_ms.item() * 1e-3) / 1e12
+    e2e_value = whole_job_tflops(world, args.steps, f_fwd + f_bwd, e2e_ms)
     tensor_bytes = B * N * H * d * 2
 
     peaks, peak_kind = load_peaks()

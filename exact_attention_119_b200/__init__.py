@@ -56,6 +56,8 @@ def library() -> ctypes.CDLL:
         lib.fa_bwd.restype = i
         lib.fa_check_device_status.argtypes = [vp]
         lib.fa_check_device_status.restype = i
+        lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+        lib.fa_bwd_noalloc.restype = i
         lib.fa_selftest_bounded_wait.argtypes = [i, i, vp]
         lib.fa_selftest_bounded_wait.restype = i
         lib.fa_status_string.argtypes = [i]
@@ -145,6 +147,39 @@ def backward(q, k, v, o, dout, lse, softmax_scale=None, causal=False, dq=None, d
     if st != FA_OK:
         raise FAError(st, "fa_bwd")
     return dq, dk, dv
+
+
+def backward_noalloc(q, k, v, o, dout, lse, softmax_scale=None, causal=False, dq=None, dk=None, dv=None,
+                     stream=None):
+    """backward() through fa_bwd_noalloc: the library's built-in scratch instead
+    of a workspace, for callers that cannot allocate device memory (the output
+    tensors are still the caller's). Calls that overlap on the GPU race on the
+    shared scratch; shapes needing more than noalloc_max_workspace() bytes of
+    scratch raise FAError (FA_ERR_WORKSPACE)."""
+    import torch
+    code = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check_bnhd(name, t, q)
+    B, N, H, d = q.shape
+    if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous [B, H, N] float32 tensor")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    st = library().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                                  lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, N, H, d,
+                                  _scale(softmax_scale, d), int(bool(causal)), code, _stream_ptr(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd_noalloc")
+    return dq, dk, dv
+
+
+# Size of the built-in scratch behind fa_bwd_noalloc (stated in include/fa.h).
+NOALLOC_MAX_WORKSPACE = 32 << 20
+
+
+def noalloc_max_workspace() -> int:
+    return NOALLOC_MAX_WORKSPACE
 
 
 def check_device_status(stream=None) -> int:

@@ -166,6 +166,40 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* 
                  : dispatch_bwd<128>(causal, bf16, mq, mk, mv, mdo, a, sms, s);
 }
 
+// ---------------------------------------------------------------------------
+// Built-in scratch for fa_bwd_noalloc.
+//
+// A file-scope device array: every GPU that loads this library holds it until
+// the process exits. In host code `g_bwd_scratch` is only a host-side stand-in
+// for the symbol, never a device address; the device address is looked up
+// with cudaGetSymbolAddress, once per device, with that device current.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) uint8_t g_bwd_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+
+// Device address of g_bwd_scratch on the current device (set up on the first
+// call for that device). Returns nullptr and sets *err on failure.
+uint8_t* noalloc_scratch(cudaError_t* err) {
+  static std::mutex mu;
+  static uint8_t* addr[kMaxDevices] = {};
+  int dev = -1;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess) return nullptr;
+  if (dev < 0 || dev >= kMaxDevices) {
+    *err = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    *err = cudaGetSymbolAddress(&p, g_bwd_scratch);
+    if (*err != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<uint8_t*>(p);
+  }
+  return addr[dev];
+}
+
 }  // namespace
 }  // namespace fa
 
@@ -216,6 +250,29 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = launch_bwd(q, k, v, o, dout, lse, dq, dk, dv, static_cast<uint8_t*>(workspace), L, B, N, H, d,
                              softmax_scale, causal != 0, dtype == FA_BF16, s);
+  if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                         const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int d,
+                         float softmax_scale, int causal, fa_dtype dtype, fa_stream_t stream) {
+  fa_status st = check_common(B, N, H, d, softmax_scale, dtype);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  const BwdLayout L = BwdLayout::make(B, N, H, d);
+  if (L.total_bytes > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;  // shape needs more than the built-in scratch
+  cudaError_t e = cudaSuccess;
+  uint8_t* scratch = noalloc_scratch(&e);
+  if (scratch == nullptr) return FA_ERR_CUDA;
+  // The preprocessing launch rewrites D and LSE*log2(e), zeroes the ordering
+  // counters and the work counter; the first key tile stores (not adds) each
+  // dQ tile. Nothing left in the scratch by an earlier call is read.
+  e = launch_bwd(q, k, v, o, dout, lse, dq, dk, dv, scratch, L, B, N, H, d, softmax_scale, causal != 0,
+                 dtype == FA_BF16, reinterpret_cast<cudaStream_t>(stream));
   if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

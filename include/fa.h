@@ -109,6 +109,35 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
                  float softmax_scale, int causal, fa_dtype dtype, fa_stream_t stream);
 
 /*
+ * fa_bwd without a workspace argument, for callers that cannot allocate
+ * device memory. The pages have no counterpart to this entry point.
+ *
+ * Some callers cannot call cudaMalloc: a plug-in or runtime whose host process
+ * owns all device memory through its own pool and allows no other allocations,
+ * code running near the device's memory capacity where a new allocation would
+ * fail, or a latency-critical loop that must not pay for the allocator. They
+ * still pass every input and output buffer; only the scratch is built in.
+ *
+ * The scratch is one file-scope device array of 32 MiB (33554432 bytes),
+ * which every GPU that loads this library holds until the process exits. No call allocates or frees device memory. A shape whose
+ * fa_bwd_workspace_size() exceeds that maximum returns FA_ERR_WORKSPACE and
+ * launches nothing.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture. All calls on a device share the one
+ * array and it keeps the last call's contents: each call re-initialises what it
+ * needs (nothing has to start at zero), but calls whose work overlaps on the
+ * GPU (different streams, or host threads, without ordering between them)
+ * race on the scratch and their results are undefined. Serialise them.
+ *
+ * Arguments, layout, results and errors are otherwise those of fa_bwd.
+ */
+FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int d,
+                                float softmax_scale, int causal, fa_dtype dtype, fa_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word of the
  * current device. Returns FA_ERR_DEVICE_TIMEOUT if any kernel of this library
  * gave up a bounded wait since the last call, FA_ERR_CUDA if the stream

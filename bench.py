@@ -72,7 +72,7 @@ def load_peaks():
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -80,17 +80,24 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.path = None
+        self.window = None
 
     def start(self):
+        """Start sampling every 50 ms; give nvidia-smi a head start."""
         try:
             import tempfile
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.5)
         except OSError:
             self.proc = None
+
+    def mark(self, t0, t1):
+        """Host wall-clock bounds of the timed region."""
+        self.window = (t0, t1)
 
     def stop(self):
         if self.proc is None:
@@ -100,26 +107,32 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        sms, maxes, reasons = [], [], set()
+        import datetime
+        sms, maxes, reasons, total = [], [], set(), 0
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
             for line in f:
                 cols = [c.strip() for c in line.split(",")]
-                if len(cols) < 9:
+                if len(cols) < 10:
                     continue
                 try:
-                    sms.append(float(cols[1]))
-                    maxes.append(float(cols[2]))
+                    ts = datetime.datetime.strptime(cols[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    sm, mx = float(cols[2]), float(cols[3])
                 except ValueError:
                     continue
-                for name, val in zip(names, cols[5:9]):
+                total += 1
+                if self.window and not (self.window[0] <= ts <= self.window[1]):
+                    continue
+                sms.append(sm)
+                maxes.append(mx)
+                for name, val in zip(names, cols[6:10]):
                     if val.lower() == "active":
                         reasons.add(name)
         os.unlink(self.path)
         if not sms:
-            return None
-        loaded = [s for s in sms if s > 0.5 * max(sms)] or sms
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(maxes), "reasons": sorted(reasons),
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": f"no sample inside the timed window ({total} outside)"}
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes), "reasons": sorted(reasons),
                 "samples": len(sms)}
 
 
@@ -210,8 +223,8 @@ def config_dict(name, workload):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -264,6 +277,7 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
         ev[i][0].record(stream)
@@ -272,6 +286,7 @@ def main():
         fa.backward(q, k, v, o, do, lse, scale, causal, dq, dk, dv, workspace=ws)
         ev[i][2].record(stream)
     torch.cuda.synchronize(dev)
+    sampler.mark(t_wall0, time.time())
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()

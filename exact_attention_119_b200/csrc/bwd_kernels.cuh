@@ -71,6 +71,7 @@ struct BwdArgs {
   int* cnt;      // [B*H, ntiles] dQ ordering counters
   int* sched;    // work counter
   int B, N, H, npad, ntiles;
+  int order;         // dQ contribution order, see BwdItem
   float scale;       // softmax_scale
   float scale_log2;  // softmax_scale * log2(e)
 };
@@ -188,8 +189,11 @@ struct BwdBarriers {
   uint64_t acc_full, acc_empty, drain;
   uint64_t item_full[2], item_empty[2];
   uint64_t dq_turn, dq_added;  // dQ warpgroup: "our turn to add", "all added"
+  uint64_t dq_rel;             // the release warp has published the step
+  uint64_t item_done;          // the release warp has published a whole item
   int item[2];
   int dq_go;     // the ordering wait succeeded
+  int dq_fail;   // some row of the step was not added (sticky)
   uint32_t tmem_base;
   int abort;
 };
@@ -221,16 +225,46 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
 }
 
 
-// Work item -> (bh, j) and the q-tile range [i_lo, ntiles).
+// Work items and the order in which key tiles add their dQ parts.
+//
+// An item is (bh, key tile j); it visits T query tiles, the s-th being
+// tile(s). For each query tile i the contributing key tiles add in one fixed
+// order; pos(i) is this item's place in it (0 = first, which stores instead of
+// adding). The orders are chosen so that, with every item of a head running at
+// once, each item's predecessor on tile i visited i one step earlier, so the
+// wait for it is already over:
+//   kCausalDesc: causal; j visits i = j, j+1, ..., n-1; tile i receives j = i,
+//                i-1, ..., 0. Items are handed out lightest first within a
+//                head (j = n-1 first), so a predecessor (j+1) always started
+//                earlier.
+//   kCyclic:     non-causal; j visits i = (j + s) mod n; tile i receives
+//                j = i, i-1, ..., 0, n-1, ..., i+1. The predecessor can have
+//                started later, so this order is only used when every item of
+//                a head fits on the grid at once (n <= grid size).
+//   kAscending:  non-causal, long sequences: j visits i = n-1, ..., 0; tile i
+//                receives j = 0, 1, ..., n-1 (the predecessor started earlier).
+enum BwdOrder : int { kCausalDesc = 0, kCyclic = 1, kAscending = 2 };
+
 struct BwdItem {
-  int bh, j, i_lo, T;
+  int bh, j, T, n, order;
+  __device__ __forceinline__ int tile(int s) const {
+    if (order == kCausalDesc) return j + s;
+    if (order == kCyclic) return (j + s) % n;
+    return n - 1 - s;
+  }
+  __device__ __forceinline__ int pos(int i) const {
+    if (order == kCausalDesc) return i - j;
+    if (order == kCyclic) return (i - j + n) % n;
+    return j;
+  }
 };
-__device__ __forceinline__ BwdItem decode_item(int item, int ntiles, bool causal) {
+__device__ __forceinline__ BwdItem decode_item(int item, int ntiles, int order) {
   BwdItem it;
   it.bh = item / ntiles;
-  it.j = item % ntiles;
-  it.i_lo = causal ? it.j : 0;
-  it.T = ntiles - it.i_lo;
+  it.j = order == kCausalDesc ? ntiles - 1 - item % ntiles : item % ntiles;
+  it.T = order == kCausalDesc ? ntiles - it.j : ntiles;
+  it.n = ntiles;
+  it.order = order;
   return it;
 }
 
@@ -258,7 +292,7 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(&bars->qdo_full[s], 1);
       mbar_init(&bars->qdo_empty[s], 1);
       mbar_init(&bars->item_full[s], 1);
-      mbar_init(&bars->item_empty[s], 13);  // MMA thread + 8 compute warps + 4 dQ warps
+      mbar_init(&bars->item_empty[s], 14);  // MMA + 8 compute warps + 4 dQ warps + release warp
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->dp_full, 1);
@@ -272,6 +306,9 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(&bars->drain, 1);
     mbar_init(&bars->dq_turn, 1);
     mbar_init(&bars->dq_added, 128);
+    mbar_init(&bars->dq_rel, 1);
+    mbar_init(&bars->item_done, 1);
+    bars->dq_fail = 0;
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -302,16 +339,20 @@ __global__ void __launch_bounds__(512, 1)
       while (ok) {
         const int slot = n_item & 1;
         if (n_item >= 2) ok = mbar_wait(&bars->item_empty[slot], ((n_item >> 1) & 1) ^ 1, abort);
+        // The cyclic order relies on every item of a head running at once, so
+        // there no item may wait in this CTA's queue behind an unfinished one:
+        // take the next item only when the previous one is fully published.
+        if (ok && a.order == kCyclic && n_item >= 1) ok = mbar_wait(&bars->item_done, (n_item - 1) & 1, abort);
         if (!ok) break;
         const int item = atomicAdd(a.sched, 1);
         bars->item[slot] = item < total_items ? item : -1;
         mbar_arrive(&bars->item_full[slot]);
         if (item >= total_items) break;
-        const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
+        const BwdItem w = decode_item(item, a.ntiles, a.order);
         const int b = w.bh / a.H, h = w.bh % a.H;
         for (int k = 0; k < w.T && ok; ++k) {
           const int st = g & 1;
-          const int i = a.ntiles - 1 - k;
+          const int i = w.tile(k);
           if (g >= 2) ok = mbar_wait(&bars->qdo_empty[st], ((g >> 1) & 1) ^ 1, abort);
           if (!ok) break;
           mbar_arrive_expect_tx(&bars->qdo_full[st], 2 * C::kTile + 1024);
@@ -375,7 +416,7 @@ __global__ void __launch_bounds__(512, 1)
         const int item = bars->item[slot];
         mbar_arrive(&bars->item_empty[slot]);
         if (item < 0) break;
-        const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
+        const BwdItem w = decode_item(item, a.ntiles, a.order);
         ok = mbar_wait(&bars->kv_full, n_item & 1, abort) && mbar_wait(&bars->qdo_full[g & 1], (g >> 1) & 1, abort);
         if (!ok) break;
         tc_fence_after();
@@ -431,6 +472,32 @@ __global__ void __launch_bounds__(512, 1)
       }
       mma_commit(&bars->drain);
       mbar_wait(&bars->drain, 0, abort, false);
+    } else if (warp == 14 && lane == 0) {
+      // ------------------------------------------------------- release warp
+      // Publishes each step's dQ additions: waits until all 128 rows of the
+      // step are in (CTA-scope acquire), then one gpu-scope release store of
+      // the tile's counter lets the next contributor add.
+      int g = 0, n_item = 0;
+      bool ok = true;
+      while (ok) {
+        const int slot = n_item & 1;
+        ok = mbar_wait(&bars->item_full[slot], (n_item >> 1) & 1, abort);
+        if (!ok) break;
+        const int item = bars->item[slot];
+        mbar_arrive(&bars->item_empty[slot]);
+        if (item < 0) break;
+        const BwdItem w = decode_item(item, a.ntiles, a.order);
+        for (int k = 0; k < w.T; ++k, ++g) {
+          const int i = w.tile(k);
+          if (!mbar_wait(&bars->dq_added, g & 1, abort)) { ok = false; break; }
+          if (bars->dq_fail) { ok = false; break; }
+          st_release(a.cnt + (size_t)w.bh * a.ntiles + i, w.pos(i) + 1);
+          mbar_arrive(&bars->dq_rel);
+        }
+        if (!ok) break;
+        mbar_arrive(&bars->item_done);
+        ++n_item;
+      }
     }
   } else if (warp < 8) {
     reg_alloc_dec<120>();
@@ -455,11 +522,11 @@ __global__ void __launch_bounds__(512, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->item_empty[slot]);
       if (item < 0) break;
-      const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
+      const BwdItem w = decode_item(item, a.ntiles, a.order);
       const int key = w.j * 128 + c;
       for (int k = 0; k < w.T; ++k, ++g) {
         const int st = g & 1;
-        const int i = a.ntiles - 1 - k;
+        const int i = w.tile(k);
         const bool diag = CAUSAL && i == w.j;
         // ---- P^T = exp2(S^T * c - LSE2) for this thread's 64 queries
         if (!mbar_wait_warp(&bars->s_full, g & 1, abort)) { ok = false; break; }
@@ -569,9 +636,9 @@ __global__ void __launch_bounds__(512, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->item_empty[slot]);
       if (item < 0) break;
-      const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
+      const BwdItem w = decode_item(item, a.ntiles, a.order);
       for (int k = 0; k < w.T; ++k, ++g) {
-        const int i = a.ntiles - 1 - k;
+        const int i = w.tile(k);
         // The warpgroup synchronises through two mbarriers (bounded waits, no
         // named barriers), so a warp that gives up cannot strand the others.
         const bool got = mbar_wait_warp(&bars->dq_full, g & 1, abort);
@@ -586,16 +653,19 @@ __global__ void __launch_bounds__(512, 1)
           tc_fence_before();
           mbar_arrive(&bars->dq_empty);
         }
-        // Thread 256 waits until key tile j-1 of this head has added its part
-        // of tile i, then opens the turn for the warpgroup.
+        // Thread 256 waits until the previous contributor to tile i has
+        // added its part (and until the release warp has published this
+        // CTA's previous step), then opens the turn for the warpgroup.
         const size_t tile = (size_t)w.bh * a.ntiles + i;
-        int* cnt = a.cnt + tile;
+        const int pos = w.pos(i);
         if (threadIdx.x == 256) {
           bool go = got;
-          if (go && w.j > 0 && ld_acquire(cnt) != w.j) {
+          if (go && g > 0) go = mbar_wait(&bars->dq_rel, (g - 1) & 1, abort);
+          const int* cnt = a.cnt + tile;
+          if (go && pos > 0 && ld_acquire(cnt) != pos) {
             const uint64_t t0 = globaltimer();
             for (uint32_t n = 1;; ++n) {
-              if (ld_acquire(cnt) == w.j) break;
+              if (ld_acquire(cnt) == pos) break;
               if ((n & 63u) == 0) {
                 if (*abort) { go = false; break; }
                 if (globaltimer() - t0 > FA_WAIT_LIMIT_NS) {
@@ -605,34 +675,33 @@ __global__ void __launch_bounds__(512, 1)
                   break;
                 }
               }
-              __nanosleep(64);
+              __nanosleep(32);
             }
           }
           bars->dq_go = go ? 1 : 0;
           mbar_arrive(&bars->dq_turn);
         }
-        const bool turn = mbar_wait(&bars->dq_turn, g & 1, abort) && bars->dq_go;
+        const bool turn = __all_sync(0xffffffffu, mbar_wait(&bars->dq_turn, g & 1, abort) && bars->dq_go);
         const bool step_ok = got && turn;
         if (step_ok) {
           float* acc = a.dqacc + tile * 128 * D;
 #pragma unroll
           for (int q = 0; q < D / 4; ++q) {
             float* p4 = acc + ((size_t)q * 128 + r) * 4;
-            if (w.j == 0)
+            if (pos == 0)
               *reinterpret_cast<float4*>(p4) = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
                                                            __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
             else
               red_add_v4(p4, __uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
                          __uint_as_float(v[4 * q + 3]));
           }
-          __threadfence();
+        } else {
+          bars->dq_fail = 1;
         }
+        // No fence here: the release warp publishes the step with one
+        // gpu-scope release after all 128 rows have arrived (the arrival is a
+        // CTA-scope release, so every add is ordered before that store).
         mbar_arrive(&bars->dq_added);
-        if (threadIdx.x == 256) {
-          // Publish only when all 128 rows are in; otherwise the next key
-          // tile's wait runs out and reports the timeout.
-          if (mbar_wait(&bars->dq_added, g & 1, abort) && step_ok) st_release(cnt, w.j + 1);
-        }
         if (!step_ok) { ok = false; break; }
       }
       if (!ok) break;

@@ -188,8 +188,9 @@ struct BwdBarriers {
   uint64_t s_full, dp_full, p_ready, ds_ready, ds_free, dq_full, dq_empty;
   uint64_t acc_full, acc_empty, drain;
   uint64_t item_full[2], item_empty[2];
-  uint64_t dq_turn, dq_added;  // dQ warpgroup: "our turn to add", "all added"
-  uint64_t dq_rel;             // the release warp has published the step
+  uint64_t dq_turn;            // dQ warpgroup: "our turn to add"
+  uint64_t dq_added[4];        // step g's 128 rows are in (ring by g % 4)
+  uint64_t dq_rel[4];          // the release warp has published step g
   uint64_t item_done;          // the release warp has published a whole item
   int item[2];
   int dq_go;     // the ordering wait succeeded
@@ -305,8 +306,10 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(&bars->acc_empty, 256);
     mbar_init(&bars->drain, 1);
     mbar_init(&bars->dq_turn, 1);
-    mbar_init(&bars->dq_added, 128);
-    mbar_init(&bars->dq_rel, 1);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&bars->dq_added[q], 128);
+      mbar_init(&bars->dq_rel[q], 1);
+    }
     mbar_init(&bars->item_done, 1);
     bars->dq_fail = 0;
     bars->abort = 0;
@@ -489,10 +492,10 @@ __global__ void __launch_bounds__(512, 1)
         const BwdItem w = decode_item(item, a.ntiles, a.order);
         for (int k = 0; k < w.T; ++k, ++g) {
           const int i = w.tile(k);
-          if (!mbar_wait(&bars->dq_added, g & 1, abort)) { ok = false; break; }
+          if (!mbar_wait(&bars->dq_added[g & 3], (g >> 2) & 1, abort)) { ok = false; break; }
           if (bars->dq_fail) { ok = false; break; }
           st_release(a.cnt + (size_t)w.bh * a.ntiles + i, w.pos(i) + 1);
-          mbar_arrive(&bars->dq_rel);
+          mbar_arrive(&bars->dq_rel[g & 3]);
         }
         if (!ok) break;
         mbar_arrive(&bars->item_done);
@@ -660,7 +663,13 @@ __global__ void __launch_bounds__(512, 1)
         const int pos = w.pos(i);
         if (threadIdx.x == 256) {
           bool go = got;
-          if (go && g > 0) go = mbar_wait(&bars->dq_rel, (g - 1) & 1, abort);
+          // Publishing step g-4 must be done before step g reuses its
+          // barriers; steps g-3 .. g-1 may still be waiting for their adds
+          // to complete in L2, which is the latency this ring hides.
+          if (go && g >= 4) go = mbar_wait(&bars->dq_rel[g & 3], ((g - 4) >> 2) & 1, abort);
+          // Every thread has passed turn g-1 (its adds are issued, not
+          // necessarily complete) before turn g reuses the single turn barrier.
+          if (go && g >= 1) go = mbar_wait(&bars->dq_added[(g - 1) & 3], ((g - 1) >> 2) & 1, abort);
           const int* cnt = a.cnt + tile;
           if (go && pos > 0 && ld_acquire(cnt) != pos) {
             const uint64_t t0 = globaltimer();
@@ -701,7 +710,7 @@ __global__ void __launch_bounds__(512, 1)
         // No fence here: the release warp publishes the step with one
         // gpu-scope release after all 128 rows have arrived (the arrival is a
         // CTA-scope release, so every add is ordered before that store).
-        mbar_arrive(&bars->dq_added);
+        mbar_arrive(&bars->dq_added[g & 3]);
         if (!step_ok) { ok = false; break; }
       }
       if (!ok) break;

@@ -13,21 +13,24 @@
 //   1. fa_bwd_prep:  D and LSE*log2(e) into padded per-head arrays; zeroes the
 //                    dQ ordering counters and the work counter.
 //   2. fa_bwd_dkdv:  persistent; one CTA per SM fetches work items (b, h, key
-//                    tile j) in increasing order. Per item K_j, V_j stay in
+//                    tile j) from a global counter. Per item K_j, V_j stay in
 //                    shared memory and dK_j, dV_j accumulate in TMEM while
-//                    (Q_i, dO_i) tiles stream through a 2-stage ring for
-//                    i = last .. first (descending). Per step, five tcgen05
-//                    MMAs: S^T = K Q^T, dP^T = V dO^T, dV += P^T dO,
-//                    dQ_part = dS K, dK += dS^T Q. dQ_part is added into an
-//                    fp32 accumulator in ascending j order (a per-tile
-//                    counter says whose turn it is), so the sum is
+//                    (Q_i, dO_i) tiles stream through a 2-stage ring. Per
+//                    step, five tcgen05 MMAs: S^T = K Q^T, dP^T = V dO^T,
+//                    dV += P^T dO, dQ_part = dS K, dK += dS^T Q. dQ_part is
+//                    added into fp32 accumulators in a fixed key-tile order
+//                    (per-tile counters say whose turn it is), so the sum is
 //                    deterministic.
-//   3. fa_bwd_dq:    dQ = scale * accumulator, cast to fp16/bf16.
+//   3. fa_bwd_dq:    dQ = scale * (lower + upper accumulator), cast.
 //
-// Ordering cannot deadlock: items start in increasing index order (a global
-// atomic counter), an item only waits for the item of key tile j-1 of the
-// same head, which has a lower index and so has already started; the lowest
-// unfinished item never waits. Every wait is bounded anyway.
+// dQ order. Key tile j visits query tiles i = j, j+1, ..., n-1 and then (non-
+// causal only) 0, 1, ..., j-1. Query tile i collects two sums: the lower one
+// from j = i, i-1, ..., 0 and the upper one from j = n-1, n-2, ..., i+1, each
+// in descending j. Items are handed out in descending j within a head, so the
+// contributor a tile waits for (j+1) was fetched earlier, and in steady state
+// it visited that tile one step earlier: the wait is already over. No wait can
+// deadlock (the earliest-fetched unfinished item waits for nothing), and
+// every wait is bounded anyway.
 #pragma once
 
 #include <algorithm>
@@ -50,8 +53,8 @@ struct BwdLayout {
     size_t off = 0;
     L.off_lse2 = off;  off = up256(off + bh * L.npad * 4);
     L.off_dd = off;    off = up256(off + bh * L.npad * 4);
-    L.off_dqacc = off; off = up256(off + bh * L.npad * (size_t)d * 4);
-    L.off_cnt = off;   off = up256(off + bh * L.ntiles * 4);
+    L.off_dqacc = off; off = up256(off + 2 * bh * L.npad * (size_t)d * 4);  // lower, upper
+    L.off_cnt = off;   off = up256(off + 2 * bh * L.ntiles * 4);            // lower, upper
     L.off_sched = off; off = up256(off + 16);
     L.total_bytes = off;
     return L;
@@ -67,11 +70,10 @@ struct BwdArgs {
   uint16_t* dv;
   float* lse2;   // [B*H, npad] LSE * log2(e); +inf on pad rows
   float* dd;     // [B*H, npad] D; 0 on pad rows
-  float* dqacc;  // [B*H, ntiles, d/4, 128, 4] fp32
-  int* cnt;      // [B*H, ntiles] dQ ordering counters
+  float* dqacc;  // 2 x [B*H, ntiles, d/4, 128, 4] fp32 (lower, upper sums)
+  int* cnt;      // 2 x [B*H, ntiles] dQ ordering counters (lower, upper)
   int* sched;    // work counter
   int B, N, H, npad, ntiles;
-  int order;         // dQ contribution order, see BwdItem
   float scale;       // softmax_scale
   float scale_log2;  // softmax_scale * log2(e)
 };
@@ -127,14 +129,14 @@ __global__ void __launch_bounds__(256) fa_bwd_prep(const BwdArgs a) {
     a.dd[bh * a.npad + n] = 0.f;
     a.lse2[bh * a.npad + n] = INFINITY;
   }
-  const long long ncnt = (long long)a.B * a.H * a.ntiles;
+  const long long ncnt = 2LL * a.B * a.H * a.ntiles;
   for (long long p = tid; p < ncnt; p += nthreads) a.cnt[p] = 0;
   if (tid == 0) *a.sched = 0;
 }
 
 // ------------------------------------------------------------------ kernel 3
 
-template <int D, bool BF16>
+template <int D, bool CAUSAL, bool BF16>
 __global__ void __launch_bounds__(256) fa_bwd_dq(const BwdArgs a) {
   // Thread per (row, 4 columns); consecutive threads take consecutive rows of
   // one tile so the accumulator reads are contiguous.
@@ -149,7 +151,15 @@ __global__ void __launch_bounds__(256) fa_bwd_dq(const BwdArgs a) {
     const long long bh = rest / a.ntiles;
     const int n = tile * 128 + r;
     if (n >= a.N) continue;
-    const float4 v = reinterpret_cast<const float4*>(a.dqacc)[t];
+    float4 v = reinterpret_cast<const float4*>(a.dqacc)[t];
+    if (!CAUSAL && tile < a.ntiles - 1) {
+      // Upper sum (key tiles after this query tile): present unless i = n-1.
+      const float4 u = reinterpret_cast<const float4*>(a.dqacc)[t + total];
+      v.x += u.x;
+      v.y += u.y;
+      v.z += u.z;
+      v.w += u.w;
+    }
     const int b = (int)(bh / a.H), h = (int)(bh % a.H);
     uint16_t* dst = a.dq + (((size_t)b * a.N + n) * a.H + h) * D + c4 * 4;
     uint2 w;
@@ -191,7 +201,6 @@ struct BwdBarriers {
   uint64_t dq_turn;            // dQ warpgroup: "our turn to add"
   uint64_t dq_added[4];        // step g's 128 rows are in (ring by g % 4)
   uint64_t dq_rel[4];          // the release warp has published step g
-  uint64_t item_done;          // the release warp has published a whole item
   int item[2];
   int dq_go;     // the ordering wait succeeded
   int dq_fail;   // some row of the step was not added (sticky)
@@ -226,46 +235,22 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
 }
 
 
-// Work items and the order in which key tiles add their dQ parts.
-//
-// An item is (bh, key tile j); it visits T query tiles, the s-th being
-// tile(s). For each query tile i the contributing key tiles add in one fixed
-// order; pos(i) is this item's place in it (0 = first, which stores instead of
-// adding). The orders are chosen so that, with every item of a head running at
-// once, each item's predecessor on tile i visited i one step earlier, so the
-// wait for it is already over:
-//   kCausalDesc: causal; j visits i = j, j+1, ..., n-1; tile i receives j = i,
-//                i-1, ..., 0. Items are handed out lightest first within a
-//                head (j = n-1 first), so a predecessor (j+1) always started
-//                earlier.
-//   kCyclic:     non-causal; j visits i = (j + s) mod n; tile i receives
-//                j = i, i-1, ..., 0, n-1, ..., i+1. The predecessor can have
-//                started later, so this order is only used when every item of
-//                a head fits on the grid at once (n <= grid size).
-//   kAscending:  non-causal, long sequences: j visits i = n-1, ..., 0; tile i
-//                receives j = 0, 1, ..., n-1 (the predecessor started earlier).
-enum BwdOrder : int { kCausalDesc = 0, kCyclic = 1, kAscending = 2 };
-
+// Work item (bh, key tile j); the s-th query tile it visits is tile(s). For
+// query tile i it adds into the lower sum (chain 0) when i >= j and into the
+// upper sum (chain 1) when i < j; pos(i) is its place in that chain's order
+// (0 = first, which stores instead of adding).
 struct BwdItem {
-  int bh, j, T, n, order;
-  __device__ __forceinline__ int tile(int s) const {
-    if (order == kCausalDesc) return j + s;
-    if (order == kCyclic) return (j + s) % n;
-    return n - 1 - s;
-  }
-  __device__ __forceinline__ int pos(int i) const {
-    if (order == kCausalDesc) return i - j;
-    if (order == kCyclic) return (i - j + n) % n;
-    return j;
-  }
+  int bh, j, T, n;
+  __device__ __forceinline__ int tile(int s) const { return j + s < n ? j + s : j + s - n; }
+  __device__ __forceinline__ int chain(int i) const { return i >= j ? 0 : 1; }
+  __device__ __forceinline__ int pos(int i) const { return i >= j ? i - j : n - 1 - j; }
 };
-__device__ __forceinline__ BwdItem decode_item(int item, int ntiles, int order) {
+__device__ __forceinline__ BwdItem decode_item(int item, int ntiles, bool causal) {
   BwdItem it;
   it.bh = item / ntiles;
-  it.j = order == kCausalDesc ? ntiles - 1 - item % ntiles : item % ntiles;
-  it.T = order == kCausalDesc ? ntiles - it.j : ntiles;
+  it.j = ntiles - 1 - item % ntiles;  // descending j within a head
+  it.T = causal ? ntiles - it.j : ntiles;
   it.n = ntiles;
-  it.order = order;
   return it;
 }
 
@@ -310,7 +295,6 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(&bars->dq_added[q], 128);
       mbar_init(&bars->dq_rel[q], 1);
     }
-    mbar_init(&bars->item_done, 1);
     bars->dq_fail = 0;
     bars->abort = 0;
     fence_mbar_init();
@@ -342,16 +326,12 @@ __global__ void __launch_bounds__(512, 1)
       while (ok) {
         const int slot = n_item & 1;
         if (n_item >= 2) ok = mbar_wait(&bars->item_empty[slot], ((n_item >> 1) & 1) ^ 1, abort);
-        // The cyclic order relies on every item of a head running at once, so
-        // there no item may wait in this CTA's queue behind an unfinished one:
-        // take the next item only when the previous one is fully published.
-        if (ok && a.order == kCyclic && n_item >= 1) ok = mbar_wait(&bars->item_done, (n_item - 1) & 1, abort);
         if (!ok) break;
         const int item = atomicAdd(a.sched, 1);
         bars->item[slot] = item < total_items ? item : -1;
         mbar_arrive(&bars->item_full[slot]);
         if (item >= total_items) break;
-        const BwdItem w = decode_item(item, a.ntiles, a.order);
+        const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
         const int b = w.bh / a.H, h = w.bh % a.H;
         for (int k = 0; k < w.T && ok; ++k) {
           const int st = g & 1;
@@ -419,7 +399,7 @@ __global__ void __launch_bounds__(512, 1)
         const int item = bars->item[slot];
         mbar_arrive(&bars->item_empty[slot]);
         if (item < 0) break;
-        const BwdItem w = decode_item(item, a.ntiles, a.order);
+        const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
         ok = mbar_wait(&bars->kv_full, n_item & 1, abort) && mbar_wait(&bars->qdo_full[g & 1], (g >> 1) & 1, abort);
         if (!ok) break;
         tc_fence_after();
@@ -489,16 +469,15 @@ __global__ void __launch_bounds__(512, 1)
         const int item = bars->item[slot];
         mbar_arrive(&bars->item_empty[slot]);
         if (item < 0) break;
-        const BwdItem w = decode_item(item, a.ntiles, a.order);
+        const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
         for (int k = 0; k < w.T; ++k, ++g) {
           const int i = w.tile(k);
           if (!mbar_wait(&bars->dq_added[g & 3], (g >> 2) & 1, abort)) { ok = false; break; }
           if (bars->dq_fail) { ok = false; break; }
-          st_release(a.cnt + (size_t)w.bh * a.ntiles + i, w.pos(i) + 1);
+          st_release(a.cnt + (size_t)w.chain(i) * a.B * a.H * a.ntiles + (size_t)w.bh * a.ntiles + i, w.pos(i) + 1);
           mbar_arrive(&bars->dq_rel[g & 3]);
         }
         if (!ok) break;
-        mbar_arrive(&bars->item_done);
         ++n_item;
       }
     }
@@ -525,7 +504,7 @@ __global__ void __launch_bounds__(512, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->item_empty[slot]);
       if (item < 0) break;
-      const BwdItem w = decode_item(item, a.ntiles, a.order);
+      const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
       const int key = w.j * 128 + c;
       for (int k = 0; k < w.T; ++k, ++g) {
         const int st = g & 1;
@@ -639,7 +618,7 @@ __global__ void __launch_bounds__(512, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->item_empty[slot]);
       if (item < 0) break;
-      const BwdItem w = decode_item(item, a.ntiles, a.order);
+      const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
       for (int k = 0; k < w.T; ++k, ++g) {
         const int i = w.tile(k);
         // The warpgroup synchronises through two mbarriers (bounded waits, no
@@ -659,7 +638,8 @@ __global__ void __launch_bounds__(512, 1)
         // Thread 256 waits until the previous contributor to tile i has
         // added its part (and until the release warp has published this
         // CTA's previous step), then opens the turn for the warpgroup.
-        const size_t tile = (size_t)w.bh * a.ntiles + i;
+        const size_t chain_off = (size_t)w.chain(i) * a.B * a.H * a.ntiles;
+        const size_t tile = (size_t)w.bh * a.ntiles + i + chain_off;
         const int pos = w.pos(i);
         if (threadIdx.x == 256) {
           bool go = got;
@@ -747,7 +727,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
   if (e != cudaSuccess) return e;
   const long long dq_threads = (long long)a.B * a.H * a.npad * (D / 4);
   const int dq_blocks = (int)std::min<long long>((dq_threads + 255) / 256, 64LL * num_sms);
-  fa_bwd_dq<D, BF16><<<dq_blocks, 256, 0, s>>>(a);
+  fa_bwd_dq<D, CAUSAL, BF16><<<dq_blocks, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 

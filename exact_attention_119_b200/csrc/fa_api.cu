@@ -160,10 +160,6 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* 
   a.H = H;
   a.npad = L.npad;
   a.ntiles = L.ntiles;
-  // dQ contribution order (see BwdItem): the cyclic order needs every key
-  // tile of a head resident at once, i.e. ntiles <= the persistent grid.
-  const int grid = std::min(B * H * L.ntiles, sms);
-  a.order = causal ? kCausalDesc : (L.ntiles <= grid ? kCyclic : kAscending);
   a.scale = scale;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634);
   return d == 64 ? dispatch_bwd<64>(causal, bf16, mq, mk, mv, mdo, a, sms, s)

@@ -177,25 +177,34 @@ struct BwdCfg {
   static constexpr int kBox = 128 * 128;     // one 64-column box of a tile
   static constexpr int kK = 0;
   static constexpr int kV = kK + kTile;
-  static constexpr int kQ = kV + kTile;            // 2 stages
-  static constexpr int kDO = kQ + 2 * kTile;       // 2 stages
-  static constexpr int kDS = kDO + 2 * kTile;      // dS^T, 128 x 128 16-bit
-  static constexpr int kLSE = kDS + 128 * 128 * 2; // 2 stages x 128 fp32
-  static constexpr int kDD = kLSE + 2 * 512;       // 2 stages x 128 fp32
-  static constexpr int kBar = kDD + 2 * 512;
+  // (Q_i, dO_i, LSE_i, D_i) ring depth: 4 stages fit at d = 64 and hide the
+  // L2 latency of the next tiles; at d = 128 shared memory allows 2.
+  static constexpr int kStages = D == 64 ? 4 : 2;
+  static constexpr int kQ = kV + kTile;                  // kStages stages
+  static constexpr int kDO = kQ + kStages * kTile;       // kStages stages
+  static constexpr int kDS = kDO + kStages * kTile;      // dS^T, 128 x 128 16-bit
+  static constexpr int kLSE = kDS + 128 * 128 * 2;       // kStages x 128 fp32
+  static constexpr int kDD = kLSE + kStages * 512;       // kStages x 128 fp32
+  static constexpr int kBar = kDD + kStages * 512;
   static constexpr int kSmem = kBar + 384;
   // TMEM columns
   static constexpr uint32_t kTdV = 0;
   static constexpr uint32_t kTdK = D;
   static constexpr uint32_t kTS = 2 * D;        // S^T, then P^T (16-bit) in place
-  static constexpr uint32_t kTdP = 2 * D + 128; // dP^T, then the dQ partial
+  static constexpr uint32_t kTdP = 2 * D + 128; // dP^T
+  // The dQ partial: at d = 64 two buffers of its own in the free columns, so
+  // the next dP^T never waits for the dQ warps; at d = 128 TMEM is full and
+  // it reuses dP^T's columns once the compute warps have read them.
+  static constexpr int kDqBufs = D == 64 ? 2 : 1;
+  __host__ __device__ static constexpr uint32_t tdq(int b) { return D == 64 ? 384u + 64u * b : kTdP; }
   static constexpr int kThreads = 512;
 };
 
 struct BwdBarriers {
   uint64_t kv_full, kv_empty;
-  uint64_t qdo_full[2], qdo_empty[2];
-  uint64_t s_full, dp_full, p_ready, ds_ready, ds_free, dq_full, dq_empty;
+  uint64_t qdo_full[4], qdo_empty[4];
+  uint64_t s_full, dp_full, p_ready, ds_ready, ds_free;
+  uint64_t dq_full[2], dq_empty[2];  // per dQ-partial buffer
   uint64_t acc_full, acc_empty, drain;
   uint64_t item_full[2], item_empty[2];
   uint64_t dq_turn;            // dQ warpgroup: "our turn to add"
@@ -274,9 +283,11 @@ __global__ void __launch_bounds__(512, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
     mbar_init(&bars->kv_empty, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&bars->qdo_full[s], 1);
       mbar_init(&bars->qdo_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->item_full[s], 1);
       mbar_init(&bars->item_empty[s], 14);  // MMA + 8 compute warps + 4 dQ warps + release warp
     }
@@ -285,8 +296,10 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(&bars->p_ready, 256);
     mbar_init(&bars->ds_ready, 256);
     mbar_init(&bars->ds_free, 1);
-    mbar_init(&bars->dq_full, 1);
-    mbar_init(&bars->dq_empty, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->dq_full[b], 1);
+      mbar_init(&bars->dq_empty[b], 128);
+    }
     mbar_init(&bars->acc_full, 1);
     mbar_init(&bars->acc_empty, 256);
     mbar_init(&bars->drain, 1);
@@ -334,9 +347,9 @@ __global__ void __launch_bounds__(512, 1)
         const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
         const int b = w.bh / a.H, h = w.bh % a.H;
         for (int k = 0; k < w.T && ok; ++k) {
-          const int st = g & 1;
+          const int st = g % C::kStages;
           const int i = w.tile(k);
-          if (g >= 2) ok = mbar_wait(&bars->qdo_empty[st], ((g >> 1) & 1) ^ 1, abort);
+          if (g >= C::kStages) ok = mbar_wait(&bars->qdo_empty[st], ((g / C::kStages) & 1) ^ 1, abort);
           if (!ok) break;
           mbar_arrive_expect_tx(&bars->qdo_full[st], 2 * C::kTile + 1024);
           for (int kb = 0; kb < D / 64; ++kb) {
@@ -365,7 +378,8 @@ __global__ void __launch_bounds__(512, 1)
       }
       // Never leave with copies in flight: the last load of each stage, and
       // the last K/V load.
-      for (int x = (g > 2 ? g - 2 : 0); x < g; ++x) mbar_wait(&bars->qdo_full[x & 1], (x >> 1) & 1, abort, false);
+      for (int x = (g > C::kStages ? g - C::kStages : 0); x < g; ++x)
+        mbar_wait(&bars->qdo_full[x % C::kStages], (x / C::kStages) & 1, abort, false);
       if (kv_loads >= 1) mbar_wait(&bars->kv_full, (kv_loads - 1) & 1, abort, false);
     } else if (warp == 13 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
@@ -400,18 +414,19 @@ __global__ void __launch_bounds__(512, 1)
         mbar_arrive(&bars->item_empty[slot]);
         if (item < 0) break;
         const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
-        ok = mbar_wait(&bars->kv_full, n_item & 1, abort) && mbar_wait(&bars->qdo_full[g & 1], (g >> 1) & 1, abort);
+        ok = mbar_wait(&bars->kv_full, n_item & 1, abort) &&
+             mbar_wait(&bars->qdo_full[g % C::kStages], (g / C::kStages) & 1, abort);
         if (!ok) break;
         tc_fence_after();
-        issue_st(dK_k, dQ_k + (g & 1) * kStage16, C::kTS);
+        issue_st(dK_k, dQ_k + (g % C::kStages) * kStage16, C::kTS);
         mma_commit(&bars->s_full);
-        if (g > 0) ok = mbar_wait(&bars->dq_empty, (g - 1) & 1, abort);
+        if (C::kDqBufs == 1 && g > 0) ok = mbar_wait(&bars->dq_empty[0], (g - 1) & 1, abort);
         if (!ok) break;
         tc_fence_after();
-        issue_st(dV_k, dDO_k + (g & 1) * kStage16, C::kTdP);
+        issue_st(dV_k, dDO_k + (g % C::kStages) * kStage16, C::kTdP);
         mma_commit(&bars->dp_full);
         for (int k = 0; k < w.T && ok; ++k, ++g) {
-          const int st = g & 1;
+          const int st = g % C::kStages;
           ok = mbar_wait(&bars->p_ready, g & 1, abort);
           if (ok && k == 0 && n_item > 0) ok = mbar_wait(&bars->acc_empty, (n_item - 1) & 1, abort);
           if (!ok) break;
@@ -422,18 +437,22 @@ __global__ void __launch_bounds__(512, 1)
             mma_ts(tmem + C::kTdV, tmem + C::kTS + kk * 8 + (kk >= 4 ? 32 : 0), dDO_mn + st * kStage16 + mstep(kk),
                    kIdKM, (k > 0 || kk > 0));
           if (k + 1 < w.T) {
-            ok = mbar_wait(&bars->qdo_full[(g + 1) & 1], ((g + 1) >> 1) & 1, abort);
+            ok = mbar_wait(&bars->qdo_full[(g + 1) % C::kStages], ((g + 1) / C::kStages) & 1, abort);
             if (!ok) break;
-            issue_st(dK_k, dQ_k + ((g + 1) & 1) * kStage16, C::kTS);
+            issue_st(dK_k, dQ_k + ((g + 1) % C::kStages) * kStage16, C::kTS);
             mma_commit(&bars->s_full);
           }
           ok = mbar_wait(&bars->ds_ready, g & 1, abort);
+          // With two dQ buffers, buffer g % 2 is free once the dQ warps have
+          // read step g - 2 out of it.
+          if (ok && C::kDqBufs == 2 && g >= 2) ok = mbar_wait(&bars->dq_empty[g & 1], ((g >> 1) & 1) ^ 1, abort);
           if (!ok) break;
           tc_fence_after();
           // dQ_part = dS K   (A = dS: dS^T stored [key][query] -> MN-major)
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) mma_ss(tmem + C::kTdP, dDS_mn + mstep(kk), dK_mn + mstep(kk), kIdQ, kk > 0);
-          mma_commit(&bars->dq_full);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + C::tdq(g % C::kDqBufs), dDS_mn + mstep(kk), dK_mn + mstep(kk), kIdQ, kk > 0);
+          mma_commit(&bars->dq_full[g % C::kDqBufs]);
           // dK += dS^T Q   (A = dS^T K-major)
 #pragma unroll
           for (int kq = 0; kq < 8; ++kq)
@@ -441,10 +460,10 @@ __global__ void __launch_bounds__(512, 1)
           mma_commit(&bars->ds_free);
           mma_commit(&bars->qdo_empty[st]);
           if (k + 1 < w.T) {
-            ok = mbar_wait(&bars->dq_empty, g & 1, abort);
+            if (C::kDqBufs == 1) ok = mbar_wait(&bars->dq_empty[0], g & 1, abort);
             if (!ok) break;
             tc_fence_after();
-            issue_st(dV_k, dDO_k + ((g + 1) & 1) * kStage16, C::kTdP);
+            issue_st(dV_k, dDO_k + ((g + 1) % C::kStages) * kStage16, C::kTdP);
             mma_commit(&bars->dp_full);
           }
         }
@@ -507,7 +526,7 @@ __global__ void __launch_bounds__(512, 1)
       const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
       const int key = w.j * 128 + c;
       for (int k = 0; k < w.T; ++k, ++g) {
-        const int st = g & 1;
+        const int st = g % C::kStages;
         const int i = w.tile(k);
         const bool diag = CAUSAL && i == w.j;
         // ---- P^T = exp2(S^T * c - LSE2) for this thread's 64 queries
@@ -515,17 +534,22 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_after();
         // P^T of queries [64 wg, 64 wg + 64), packed two per 32-bit word.
         uint32_t pk[32];
+        uint32_t sv[64];
+        tmem_ld32(lane_base + C::kTS + wg * 64, sv);
+        tmem_ld32(lane_base + C::kTS + wg * 64 + 32, sv + 32);
+        tmem_ld_wait();
+        tie_regs32(sv);
+        tie_regs32(sv + 32);
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
-          uint32_t s[32];
-          tmem_ld32(lane_base + C::kTS + wg * 64 + h2 * 32, s);
-          tmem_ld_wait();
-          tie_regs32(s);
+          const uint32_t* s = sv + h2 * 32;
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
             const int qc = wg * 64 + h2 * 32 + 2 * x;
-            float v0 = ex2(fmaf(__uint_as_float(s[2 * x]), cl2, -sLSE[st * 128 + qc]));
-            float v1 = ex2(fmaf(__uint_as_float(s[2 * x + 1]), cl2, -sLSE[st * 128 + qc + 1]));
+            // LSE*log2(e) of these two query columns (one 8-byte broadcast load)
+            const float2 l2 = *reinterpret_cast<const float2*>(sLSE + st * 128 + qc);
+            float v0 = ex2(fmaf(__uint_as_float(s[2 * x]), cl2, -l2.x));
+            float v1 = ex2(fmaf(__uint_as_float(s[2 * x + 1]), cl2, -l2.y));
             if (diag && key > i * 128 + qc) v0 = 0.f;
             if (diag && key > i * 128 + qc + 1) v1 = 0.f;
             pk[h2 * 16 + x] = pack2<BF16>(v0, v1);
@@ -553,8 +577,9 @@ __global__ void __launch_bounds__(512, 1)
           for (int x = 0; x < 16; ++x) {
             const int qc = wg * 64 + h2 * 32 + 2 * x;
             const float2 pp = unpack2<BF16>(pk[h2 * 16 + x]);
-            const float d0 = pp.x * (__uint_as_float(dp[2 * x]) - sDD[st * 128 + qc]);
-            const float d1 = pp.y * (__uint_as_float(dp[2 * x + 1]) - sDD[st * 128 + qc + 1]);
+            const float2 dd = *reinterpret_cast<const float2*>(sDD + st * 128 + qc);
+            const float d0 = pp.x * (__uint_as_float(dp[2 * x]) - dd.x);
+            const float d1 = pp.y * (__uint_as_float(dp[2 * x + 1]) - dd.y);
             dsk[x] = pack2<BF16>(d0, d1);
           }
           // Row c of a 128-byte-swizzled [128][64] box: 16-byte chunk x goes
@@ -607,7 +632,7 @@ __global__ void __launch_bounds__(512, 1)
     // Thread = query row r of the step (TMEM lane).
     const int quad = warp % 4;
     const int r = quad * 32 + lane;
-    const uint32_t src = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::kTdP;
+    const uint32_t src0 = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     int g = 0, n_item = 0;
     bool ok = true;
     while (ok) {
@@ -623,7 +648,9 @@ __global__ void __launch_bounds__(512, 1)
         const int i = w.tile(k);
         // The warpgroup synchronises through two mbarriers (bounded waits, no
         // named barriers), so a warp that gives up cannot strand the others.
-        const bool got = mbar_wait_warp(&bars->dq_full, g & 1, abort);
+        const int buf = g % C::kDqBufs;
+        const uint32_t src = src0 + C::tdq(buf);
+        const bool got = mbar_wait_warp(&bars->dq_full[buf], (g / C::kDqBufs) & 1, abort);
         uint32_t v[D];
         if (got) {
           tc_fence_after();
@@ -633,7 +660,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
           for (int q = 0; q < D / 32; ++q) tie_regs32(v + q * 32);
           tc_fence_before();
-          mbar_arrive(&bars->dq_empty);
+          mbar_arrive(&bars->dq_empty[buf]);
         }
         // Thread 256 waits until the previous contributor to tile i has
         // added its part (and until the release warp has published this

@@ -18,6 +18,12 @@
 // The two tiles ping-pong: while one softmax warpgroup works on its S, the
 // tensor core runs the other tile's P V and next S.
 //
+// At d = 64 TMEM has room for P next to S (kSepP): the softmax signals "S
+// consumed" as soon as S is in registers, so S of the next key tile is
+// computed while the softmax is still busy with exponentials, and the
+// exponential unit is not left idle waiting for the next S. At d = 128 P
+// overwrites S in place and the next S follows P V.
+//
 // Online softmax with a lagging reference max: the running max m (log2
 // units) is only moved, and O and l rescaled, when a tile's max exceeds m by
 // more than kRescaleLog2 (so P <= 2^kRescaleLog2). The final O / l and
@@ -49,9 +55,12 @@ struct FwdCfg {
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
   static constexpr int kSmemBytes = kBarOff + 512 + 1024;  // + barriers + alignment slack
-  // TMEM columns: S/P of tile t at tmem_s(t), O of tile t at tmem_o(t).
+  // TMEM columns: S of tile t at tmem_s(t), O at tmem_o(t), P at tmem_p(t)
+  // (its own 64 columns when kSepP, else over S).
+  static constexpr bool kSepP = D == 64;
   __host__ __device__ static constexpr uint32_t tmem_s(int t) { return t ? 128u : 0u; }
   __host__ __device__ static constexpr uint32_t tmem_o(int t) { return t ? 256u + D : 256u; }
+  __host__ __device__ static constexpr uint32_t tmem_p(int t) { return kSepP ? 384u + 64u * t : tmem_s(t); }
   static constexpr int kThreads = 384;
 };
 
@@ -60,6 +69,8 @@ struct FwdBarriers {
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_full[2];
+  uint64_t s_cons[2];   // kSepP: the softmax has S(t, j) in registers
+  uint64_t pv_done[2];  // kSepP: P(t, j) V_j has completed
   uint64_t drain;
   uint64_t kv_full[8];
   uint64_t kv_empty[8];
@@ -98,6 +109,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bars->s_full[t], 1);
       mbar_init(&bars->p_full[t], 128);
       mbar_init(&bars->o_full[t], 1);
+      mbar_init(&bars->s_cons[t], 128);
+      mbar_init(&bars->pv_done[t], 1);
     }
     mbar_init(&bars->drain, 1);
     for (int s = 0; s < C::kStages; ++s) {
@@ -180,51 +193,90 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t va = dKV_mn + (uint64_t)(stage * kTile16);
 #pragma unroll
         for (int kk = 0; kk < C::kKeys / 16; ++kk)
-          mma_ts(tmem + C::tmem_o(t), tmem + C::tmem_s(t) + kk * 8, va + (uint64_t)(kk * (2048 >> 4)), kIdPV,
+          mma_ts(tmem + C::tmem_o(t), tmem + C::tmem_p(t) + kk * 8, va + (uint64_t)(kk * (2048 >> 4)), kIdPV,
                  (acc || kk > 0) ? 1u : 0u);
       };
       auto kv_wait = [&](int pos) { return mbar_wait(&bars->kv_full[pos % C::kStages], (pos / C::kStages) & 1, abort); };
 
       bool ok = mbar_wait(&bars->q_full, 0, abort) && kv_wait(0);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        mma_commit(&bars->s_full[0]);
-        issue_s(1, 0);
-        mma_commit(&bars->s_full[1]);
-        mma_commit(&bars->kv_empty[0]);
-      }
-      for (int j = 1; j < n_kv && ok; ++j) {
-        const int pv = 2 * j - 1, pk = 2 * j;  // ring positions of V_{j-1} and K_j
-        ok = kv_wait(pv) && kv_wait(pk) && mbar_wait(&bars->p_full[0], (j - 1) & 1, abort);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(0, pv % C::kStages, j > 1);
-        issue_s(0, pk % C::kStages);
-        mma_commit(&bars->s_full[0]);
-        ok = mbar_wait(&bars->p_full[1], (j - 1) & 1, abort);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(1, pv % C::kStages, j > 1);
-        mma_commit(&bars->kv_empty[pv % C::kStages]);
-        issue_s(1, pk % C::kStages);
-        mma_commit(&bars->s_full[1]);
-        mma_commit(&bars->kv_empty[pk % C::kStages]);
-      }
-      if (ok) {
-        const int pv = 2 * n_kv - 1;
-        ok = kv_wait(pv) && mbar_wait(&bars->p_full[0], (n_kv - 1) & 1, abort);
+      if constexpr (C::kSepP) {
+        // S(t, j+1) as soon as S(t, j) is in registers; P(t, j) V_j when P is
+        // ready. Ring positions: K_j at 2j, V_j at 2j + 1.
         if (ok) {
           tc_fence_after();
-          issue_pv(0, pv % C::kStages, n_kv > 1);
-          mma_commit(&bars->o_full[0]);
-          ok = mbar_wait(&bars->p_full[1], (n_kv - 1) & 1, abort);
+          issue_s(0, 0);
+          mma_commit(&bars->s_full[0]);
+          issue_s(1, 0);
+          mma_commit(&bars->s_full[1]);
+          mma_commit(&bars->kv_empty[0]);
+        }
+        for (int j = 0; j < n_kv && ok; ++j) {
+          if (j + 1 < n_kv) {
+            const int pk = 2 * j + 2;
+            ok = kv_wait(pk);
+            for (int t = 0; t < 2 && ok; ++t) {
+              ok = mbar_wait(&bars->s_cons[t], j & 1, abort);
+              if (!ok) break;
+              tc_fence_after();
+              issue_s(t, pk % C::kStages);
+              mma_commit(&bars->s_full[t]);
+            }
+            if (!ok) break;
+            mma_commit(&bars->kv_empty[pk % C::kStages]);
+          }
+          const int pv = 2 * j + 1;
+          ok = kv_wait(pv);
+          for (int t = 0; t < 2 && ok; ++t) {
+            ok = mbar_wait(&bars->p_full[t], j & 1, abort);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(t, pv % C::kStages, j > 0);
+            mma_commit(j + 1 < n_kv ? &bars->pv_done[t] : &bars->o_full[t]);
+          }
+          if (!ok) break;
+          mma_commit(&bars->kv_empty[pv % C::kStages]);
+        }
+      } else {
+        if (ok) {
+          tc_fence_after();
+          issue_s(0, 0);
+          mma_commit(&bars->s_full[0]);
+          issue_s(1, 0);
+          mma_commit(&bars->s_full[1]);
+          mma_commit(&bars->kv_empty[0]);
+        }
+        for (int j = 1; j < n_kv && ok; ++j) {
+          const int pv = 2 * j - 1, pk = 2 * j;  // ring positions of V_{j-1} and K_j
+          ok = kv_wait(pv) && kv_wait(pk) && mbar_wait(&bars->p_full[0], (j - 1) & 1, abort);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(0, pv % C::kStages, j > 1);
+          issue_s(0, pk % C::kStages);
+          mma_commit(&bars->s_full[0]);
+          ok = mbar_wait(&bars->p_full[1], (j - 1) & 1, abort);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(1, pv % C::kStages, j > 1);
+          mma_commit(&bars->kv_empty[pv % C::kStages]);
+          issue_s(1, pk % C::kStages);
+          mma_commit(&bars->s_full[1]);
+          mma_commit(&bars->kv_empty[pk % C::kStages]);
         }
         if (ok) {
-          tc_fence_after();
-          issue_pv(1, pv % C::kStages, n_kv > 1);
-          mma_commit(&bars->o_full[1]);
-          mma_commit(&bars->kv_empty[pv % C::kStages]);
+          const int pv = 2 * n_kv - 1;
+          ok = kv_wait(pv) && mbar_wait(&bars->p_full[0], (n_kv - 1) & 1, abort);
+          if (ok) {
+            tc_fence_after();
+            issue_pv(0, pv % C::kStages, n_kv > 1);
+            mma_commit(&bars->o_full[0]);
+            ok = mbar_wait(&bars->p_full[1], (n_kv - 1) & 1, abort);
+          }
+          if (ok) {
+            tc_fence_after();
+            issue_pv(1, pv % C::kStages, n_kv > 1);
+            mma_commit(&bars->o_full[1]);
+            mma_commit(&bars->kv_empty[pv % C::kStages]);
+          }
         }
       }
       // Every issued MMA has finished before the CTA may release TMEM.
@@ -260,6 +312,10 @@ __global__ void __launch_bounds__(384, 1)
       tmem_ld_wait();
 #pragma unroll
       for (int q = 0; q < 4; ++q) tie_regs32(s + q * 32);
+      if constexpr (C::kSepP) {
+        tc_fence_before();
+        mbar_arrive(&bars->s_cons[t]);  // S(t, j+1) may now be written over S(t, j)
+      }
 
       const int kv0 = j * C::kKeys;
       if (kv0 + C::kKeys > lim) {
@@ -281,8 +337,18 @@ __global__ void __launch_bounds__(384, 1)
         m = m_tile;
         need = true;
       }
+      // kSepP: P(t, j-1) V_{j-1} must be complete before O is rescaled or P is
+      // rewritten (without kSepP its commit preceded s_full already).
+      bool pv_waited = !C::kSepP || j == 0;
       if (__any_sync(0xffffffffu, need)) {
-        // P V of the previous tile has completed (its commit preceded s_full).
+        if (!pv_waited) {
+          if (!mbar_wait_warp(&bars->pv_done[t], (j - 1) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          pv_waited = true;
+        }
 #pragma unroll 1
         for (int q = 0; q < D / 16; ++q) {
           uint32_t o[16];
@@ -297,6 +363,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       l *= alpha;
       lr *= alpha;
+      const uint32_t tP = lane_base + C::tmem_p(t);
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
       float sum = 0.f, sum_r = 0.f;
 #pragma unroll
@@ -311,8 +378,17 @@ __global__ void __launch_bounds__(384, 1)
           sum += p0 + p1;
           sum_r += r.x + r.y;
         }
-        tmem_st16(tS + part * 16, p);
+        if (part == 0 && !pv_waited) {
+          if (!mbar_wait_warp(&bars->pv_done[t], (j - 1) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          pv_waited = true;
+        }
+        tmem_st16(tP + part * 16, p);
       }
+      if (!ok) break;
       l += sum;
       lr += sum_r;
       tmem_st_wait();

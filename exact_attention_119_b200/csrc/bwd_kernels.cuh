@@ -196,6 +196,17 @@ struct BwdCfg {
   // the next dP^T never waits for the dQ warps; at d = 128 TMEM is full and
   // it reuses dP^T's columns once the compute warps have read them.
   static constexpr int kDqBufs = D == 64 ? 2 : 1;
+  // d = 64: the compute warps run one step ahead (P of step g+1 before dS of
+  // step g) and the MMA warp issues dV(g+1), S(g+2) before dQ(g), dK(g). That
+  // needs S(g+2)'s Q tile loaded before dK(g) frees a stage: kStages >= 3.
+  static constexpr bool kSkew = D == 64;
+  static_assert(!kSkew || kStages >= 3, "the skewed schedule needs a third Q/dO stage");
+  // setmaxnreg budgets per warpgroup (one warp of each on every SM
+  // sub-partition); they add up to the 4 x 128 the CTA is launched with.
+  static constexpr int kRegsProd = 112;
+  static constexpr int kRegsCompute = D == 64 ? 152 : 120;  // x 2 warpgroups
+  static constexpr int kRegsDQ = D == 64 ? 96 : 160;
+  static_assert(kRegsProd + 2 * kRegsCompute + kRegsDQ == 512, "register split must use the launch allocation");
   __host__ __device__ static constexpr uint32_t tdq(int b) { return D == 64 ? 384u + 64u * b : kTdP; }
   static constexpr int kThreads = 512;
 };
@@ -322,10 +333,10 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t tmem = bars->tmem_base;
 
   // Register split per SM sub-partition (one warp of each warpgroup on each):
-  // producer/MMA 112 + compute 120 + compute 120 + dQ 160 = 512 = the 4 x 128
-  // the CTA was launched with, so the one setmaxnreg.inc cannot wait forever.
+  // producer/MMA + 2 x compute + dQ = 512 = the 4 x 128 the CTA was launched
+  // with (BwdCfg), so no setmaxnreg.inc can wait forever.
   if (warp >= 12) {
-    reg_alloc_dec<112>();
+    reg_alloc_set<C::kRegsProd, 128>();
     if (warp == 12 && elect_one()) {
       // ------------------------------------------------------------ producer
       tma_prefetch_desc(&tm_q);
@@ -425,46 +436,112 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_after();
         issue_st(dV_k, dDO_k + (g % C::kStages) * kStage16, C::kTdP);
         mma_commit(&bars->dp_full);
-        for (int k = 0; k < w.T && ok; ++k, ++g) {
-          const int st = g % C::kStages;
+        if constexpr (C::kSkew) {
+          // Order matches the compute warps, which run one step ahead:
+          // P(g+1) arrives before dS(g).
+          auto issue_dv = [&](int gs, bool acc) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts(tmem + C::kTdV, tmem + C::kTS + kk * 8 + (kk >= 4 ? 32 : 0),
+                     dDO_mn + (gs % C::kStages) * kStage16 + mstep(kk), kIdKM, (acc || kk > 0));
+          };
           ok = mbar_wait(&bars->p_ready, g & 1, abort);
-          if (ok && k == 0 && n_item > 0) ok = mbar_wait(&bars->acc_empty, (n_item - 1) & 1, abort);
-          if (!ok) break;
-          tc_fence_after();
-          // dV += P^T dO   (A = P^T in TMEM, 16-bit packed)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + C::kTdV, tmem + C::kTS + kk * 8 + (kk >= 4 ? 32 : 0), dDO_mn + st * kStage16 + mstep(kk),
-                   kIdKM, (k > 0 || kk > 0));
-          if (k + 1 < w.T) {
-            ok = mbar_wait(&bars->qdo_full[(g + 1) % C::kStages], ((g + 1) / C::kStages) & 1, abort);
-            if (!ok) break;
-            issue_st(dK_k, dQ_k + ((g + 1) % C::kStages) * kStage16, C::kTS);
-            mma_commit(&bars->s_full);
+          if (ok && n_item > 0) ok = mbar_wait(&bars->acc_empty, (n_item - 1) & 1, abort);
+          if (ok) {
+            tc_fence_after();
+            issue_dv(g, false);
+            if (w.T > 1) {
+              ok = mbar_wait(&bars->qdo_full[(g + 1) % C::kStages], ((g + 1) / C::kStages) & 1, abort);
+              if (ok) {
+                issue_st(dK_k, dQ_k + ((g + 1) % C::kStages) * kStage16, C::kTS);
+                mma_commit(&bars->s_full);
+              }
+            }
           }
-          ok = mbar_wait(&bars->ds_ready, g & 1, abort);
-          // With two dQ buffers, buffer g % 2 is free once the dQ warps have
-          // read step g - 2 out of it.
-          if (ok && C::kDqBufs == 2 && g >= 2) ok = mbar_wait(&bars->dq_empty[g & 1], ((g >> 1) & 1) ^ 1, abort);
-          if (!ok) break;
-          tc_fence_after();
-          // dQ_part = dS K   (A = dS: dS^T stored [key][query] -> MN-major)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + C::tdq(g % C::kDqBufs), dDS_mn + mstep(kk), dK_mn + mstep(kk), kIdQ, kk > 0);
-          mma_commit(&bars->dq_full[g % C::kDqBufs]);
-          // dK += dS^T Q   (A = dS^T K-major)
-#pragma unroll
-          for (int kq = 0; kq < 8; ++kq)
-            mma_ss(tmem + C::kTdK, dDS_k + kstep(kq), dQ_mn + st * kStage16 + mstep(kq), kIdKM, (k > 0 || kq > 0));
-          mma_commit(&bars->ds_free);
-          mma_commit(&bars->qdo_empty[st]);
-          if (k + 1 < w.T) {
-            if (C::kDqBufs == 1) ok = mbar_wait(&bars->dq_empty[0], g & 1, abort);
+          for (int k = 0; k < w.T && ok; ++k, ++g) {
+            const int st = g % C::kStages;
+            if (k + 1 < w.T) {
+              ok = mbar_wait(&bars->p_ready, (g + 1) & 1, abort);
+              if (!ok) break;
+              tc_fence_after();
+              issue_dv(g + 1, true);
+              if (k + 2 < w.T) {
+                ok = mbar_wait(&bars->qdo_full[(g + 2) % C::kStages], ((g + 2) / C::kStages) & 1, abort);
+                if (!ok) break;
+                issue_st(dK_k, dQ_k + ((g + 2) % C::kStages) * kStage16, C::kTS);
+                mma_commit(&bars->s_full);
+              }
+            }
+            ok = mbar_wait(&bars->ds_ready, g & 1, abort);
             if (!ok) break;
             tc_fence_after();
-            issue_st(dV_k, dDO_k + ((g + 1) % C::kStages) * kStage16, C::kTdP);
-            mma_commit(&bars->dp_full);
+            if (k + 1 < w.T) {
+              issue_st(dV_k, dDO_k + ((g + 1) % C::kStages) * kStage16, C::kTdP);
+              mma_commit(&bars->dp_full);
+            }
+            if (g >= 2) ok = mbar_wait(&bars->dq_empty[g & 1], ((g >> 1) & 1) ^ 1, abort);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tmem + C::tdq(g & 1), dDS_mn + mstep(kk), dK_mn + mstep(kk), kIdQ, kk > 0);
+            mma_commit(&bars->dq_full[g & 1]);
+#pragma unroll
+            for (int kq = 0; kq < 8; ++kq)
+              mma_ss(tmem + C::kTdK, dDS_k + kstep(kq), dQ_mn + st * kStage16 + mstep(kq), kIdKM, (k > 0 || kq > 0));
+            mma_commit(&bars->ds_free);
+            mma_commit(&bars->qdo_empty[st]);
+          }
+        } else {
+          for (int k = 0; k < w.T && ok; ++k, ++g) {
+            const int st = g % C::kStages;
+            ok = mbar_wait(&bars->p_ready, g & 1, abort);
+            if (ok && k == 0 && n_item > 0) ok = mbar_wait(&bars->acc_empty, (n_item - 1) & 1, abort);
+            if (!ok) break;
+            tc_fence_after();
+            // dV += P^T dO   (A = P^T in TMEM, 16-bit packed)
+  #pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts(tmem + C::kTdV, tmem + C::kTS + kk * 8 + (kk >= 4 ? 32 : 0), dDO_mn + st * kStage16 + mstep(kk),
+                     kIdKM, (k > 0 || kk > 0));
+            if (k + 1 < w.T) {
+              ok = mbar_wait(&bars->qdo_full[(g + 1) % C::kStages], ((g + 1) / C::kStages) & 1, abort);
+              if (!ok) break;
+              issue_st(dK_k, dQ_k + ((g + 1) % C::kStages) * kStage16, C::kTS);
+              mma_commit(&bars->s_full);
+            }
+            ok = mbar_wait(&bars->ds_ready, g & 1, abort);
+            if (!ok) break;
+            tc_fence_after();
+            if (C::kDqBufs == 2 && k + 1 < w.T) {
+              // dP^T(g+1) has its own columns here: issue it ahead of dQ(g) and
+              // dK(g) so the compute warps' next dS phase does not queue behind them.
+              issue_st(dV_k, dDO_k + ((g + 1) % C::kStages) * kStage16, C::kTdP);
+              mma_commit(&bars->dp_full);
+            }
+            // With two dQ buffers, buffer g % 2 is free once the dQ warps have
+            // read step g - 2 out of it.
+            if (C::kDqBufs == 2 && g >= 2) ok = mbar_wait(&bars->dq_empty[g & 1], ((g >> 1) & 1) ^ 1, abort);
+            if (!ok) break;
+            tc_fence_after();
+            // dQ_part = dS K   (A = dS: dS^T stored [key][query] -> MN-major)
+  #pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tmem + C::tdq(g % C::kDqBufs), dDS_mn + mstep(kk), dK_mn + mstep(kk), kIdQ, kk > 0);
+            mma_commit(&bars->dq_full[g % C::kDqBufs]);
+            // dK += dS^T Q   (A = dS^T K-major)
+  #pragma unroll
+            for (int kq = 0; kq < 8; ++kq)
+              mma_ss(tmem + C::kTdK, dDS_k + kstep(kq), dQ_mn + st * kStage16 + mstep(kq), kIdKM, (k > 0 || kq > 0));
+            mma_commit(&bars->ds_free);
+            mma_commit(&bars->qdo_empty[st]);
+            if (C::kDqBufs == 1 && k + 1 < w.T) {
+              ok = mbar_wait(&bars->dq_empty[0], g & 1, abort);
+              if (!ok) break;
+              tc_fence_after();
+              issue_st(dV_k, dDO_k + ((g + 1) % C::kStages) * kStage16, C::kTdP);
+              mma_commit(&bars->dp_full);
+            }
           }
         }
         if (!ok) break;
@@ -501,7 +578,7 @@ __global__ void __launch_bounds__(512, 1)
       }
     }
   } else if (warp < 8) {
-    reg_alloc_dec<120>();
+    reg_alloc_set<C::kRegsCompute, 128>();
     // ------------------------------------------------------- compute warps
     // Thread = key row c (TMEM lane); warpgroup wg takes query columns
     // [64 wg, 64 wg + 64) of each 128 x 128 step.
@@ -525,46 +602,43 @@ __global__ void __launch_bounds__(512, 1)
       if (item < 0) break;
       const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
       const int key = w.j * 128 + c;
-      for (int k = 0; k < w.T; ++k, ++g) {
-        const int st = g % C::kStages;
-        const int i = w.tile(k);
+      // P^T = exp2(S^T * c - LSE2) of step gs (query tile i) for this thread's
+      // 64 queries, packed two per word into pk and written to TMEM over S^T
+      // (columns this warpgroup has already read).
+      auto p_phase = [&](int gs, int i, uint32_t* pk) -> bool {
+        const int st = gs % C::kStages;
         const bool diag = CAUSAL && i == w.j;
-        // ---- P^T = exp2(S^T * c - LSE2) for this thread's 64 queries
-        if (!mbar_wait_warp(&bars->s_full, g & 1, abort)) { ok = false; break; }
+        if (!mbar_wait_warp(&bars->s_full, gs & 1, abort)) return false;
         tc_fence_after();
-        // P^T of queries [64 wg, 64 wg + 64), packed two per 32-bit word.
-        uint32_t pk[32];
-        uint32_t sv[64];
-        tmem_ld32(lane_base + C::kTS + wg * 64, sv);
-        tmem_ld32(lane_base + C::kTS + wg * 64 + 32, sv + 32);
-        tmem_ld_wait();
-        tie_regs32(sv);
-        tie_regs32(sv + 32);
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
-          const uint32_t* s = sv + h2 * 32;
+          uint32_t sv[32];
+          tmem_ld32(lane_base + C::kTS + wg * 64 + h2 * 32, sv);
+          tmem_ld_wait();
+          tie_regs32(sv);
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
             const int qc = wg * 64 + h2 * 32 + 2 * x;
-            // LSE*log2(e) of these two query columns (one 8-byte broadcast load)
             const float2 l2 = *reinterpret_cast<const float2*>(sLSE + st * 128 + qc);
-            float v0 = ex2(fmaf(__uint_as_float(s[2 * x]), cl2, -l2.x));
-            float v1 = ex2(fmaf(__uint_as_float(s[2 * x + 1]), cl2, -l2.y));
+            float v0 = ex2(fmaf(__uint_as_float(sv[2 * x]), cl2, -l2.x));
+            float v1 = ex2(fmaf(__uint_as_float(sv[2 * x + 1]), cl2, -l2.y));
             if (diag && key > i * 128 + qc) v0 = 0.f;
             if (diag && key > i * 128 + qc + 1) v1 = 0.f;
             pk[h2 * 16 + x] = pack2<BF16>(v0, v1);
           }
         }
-        // It goes into columns [64 wg, 64 wg + 32) of S: columns this
-        // warpgroup has already read, so the other warpgroup's S is untouched.
         tmem_st32(lane_base + C::kTS + wg * 64, pk);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars->p_ready);
-        // ---- dS^T = P^T o (dP^T - D) -> shared memory (16-bit), from the same
-        // rounded P that the dV product uses.
-        if (!mbar_wait_warp(&bars->dp_full, g & 1, abort)) { ok = false; break; }
-        if (g > 0 && !mbar_wait_warp(&bars->ds_free, (g - 1) & 1, abort)) { ok = false; break; }
+        return true;
+      };
+      // dS^T = P^T o (dP^T - D) of step gs -> shared memory (16-bit), from the
+      // same rounded P that the dV product uses.
+      auto ds_phase = [&](int gs, const uint32_t* pk) -> bool {
+        const int st = gs % C::kStages;
+        if (!mbar_wait_warp(&bars->dp_full, gs & 1, abort)) return false;
+        if (gs > 0 && !mbar_wait_warp(&bars->ds_free, (gs - 1) & 1, abort)) return false;
         tc_fence_after();
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -591,9 +665,28 @@ __global__ void __launch_bounds__(512, 1)
             *dst = make_uint4(dsk[4 * x], dsk[4 * x + 1], dsk[4 * x + 2], dsk[4 * x + 3]);
           }
         }
-        tc_fence_before();  // dP^T reads done before the dQ MMA reuses these columns
+        tc_fence_before();  // dP^T reads done before the next MMA may reuse these columns
         fence_proxy_async_smem();
         mbar_arrive(&bars->ds_ready);
+        return true;
+      };
+      // Software-pipelined by one step: P of step g+1 is computed before dS
+      // of step g, so dS(g) finds dP(g) finished (it was issued a whole P
+      // phase earlier) and P(g+1) only waits for dV(g) and S(g+1).
+      if constexpr (C::kSkew) {
+        uint32_t pk_cur[32], pk_next[32];
+        if (!p_phase(g, w.tile(0), pk_cur)) { ok = false; break; }
+        for (int k = 0; k < w.T; ++k, ++g) {
+          if (k + 1 < w.T && !p_phase(g + 1, w.tile(k + 1), pk_next)) { ok = false; break; }
+          if (!ds_phase(g, pk_cur)) { ok = false; break; }
+#pragma unroll
+          for (int x = 0; x < 32; ++x) pk_cur[x] = pk_next[x];
+        }
+      } else {
+        for (int k = 0; k < w.T; ++k, ++g) {
+          uint32_t pk[32];
+          if (!p_phase(g, w.tile(k), pk) || !ds_phase(g, pk)) { ok = false; break; }
+        }
       }
       if (!ok) break;
       // ---- epilogue: warpgroup 0 stores dV_j, warpgroup 1 stores scale * dK_j
@@ -627,7 +720,7 @@ __global__ void __launch_bounds__(512, 1)
       ++n_item;
     }
   } else {
-    reg_alloc_inc<160>();
+    reg_alloc_set<C::kRegsDQ, 128>();
     // ------------------------------------------------------ dQ warps (8-11)
     // Thread = query row r of the step (TMEM lane).
     const int quad = warp % 4;

@@ -276,6 +276,13 @@ __device__ __forceinline__ void reg_alloc_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(NREG));
 }
 
+// Move this warpgroup's budget from the launch count FROM to NREG.
+template <int NREG, int FROM>
+__device__ __forceinline__ void reg_alloc_set() {
+  if constexpr (NREG > FROM) reg_alloc_inc<NREG>();
+  else if constexpr (NREG < FROM) reg_alloc_dec<NREG>();
+}
+
 // --------------------------------------------------------------- arithmetic
 
 __device__ __forceinline__ float ex2(float x) {

@@ -323,9 +323,16 @@ __global__ void __launch_bounds__(384, 1)
         for (int i = 0; i < 128; ++i)
           if (kv0 + i >= lim) s[i] = __float_as_uint(-INFINITY);
       }
-      float mx = -INFINITY;
+      // Row max: eight independent chains of three-operand max, then a tree.
+      float mxa[8];
 #pragma unroll
-      for (int i = 0; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(s[i]));
+      for (int k = 0; k < 8; ++k) {
+        float x = max3(__uint_as_float(s[k]), __uint_as_float(s[k + 8]), __uint_as_float(s[k + 16]));
+#pragma unroll
+        for (int e = 3; e + 1 < 16; e += 2) x = max3(x, __uint_as_float(s[k + 8 * e]), __uint_as_float(s[k + 8 * e + 8]));
+        mxa[k] = fmaxf(x, __uint_as_float(s[k + 120]));
+      }
+      const float mx = max3(max3(mxa[0], mxa[1], mxa[2]), max3(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]));
       const float m_tile = mx * c;
 
       float alpha = 1.f;
@@ -365,7 +372,9 @@ __global__ void __launch_bounds__(384, 1)
       lr *= alpha;
       const uint32_t tP = lane_base + C::tmem_p(t);
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
-      float sum = 0.f, sum_r = 0.f;
+      // Four accumulators each for the exact and the rounded sums, so no add
+      // waits on the one before it.
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sra[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int part = 0; part < 4; ++part) {
         uint32_t p[16];
@@ -374,9 +383,11 @@ __global__ void __launch_bounds__(384, 1)
           const float p0 = ex2(fmaf(__uint_as_float(s[part * 32 + 2 * i]), c, neg_m));
           const float p1 = ex2(fmaf(__uint_as_float(s[part * 32 + 2 * i + 1]), c, neg_m));
           p[i] = pack2<BF16>(p0, p1);
-          const float2 r = unpack2<BF16>(p[i]);
-          sum += p0 + p1;
-          sum_r += r.x + r.y;
+          const int a = 2 * (i & 1);
+          sa[a] += p0;
+          sa[a + 1] += p1;
+          sra[a] = add_lo16<BF16>(sra[a], p[i]);
+          sra[a + 1] = add_hi16<BF16>(sra[a + 1], p[i]);
         }
         if (part == 0 && !pv_waited) {
           if (!mbar_wait_warp(&bars->pv_done[t], (j - 1) & 1, abort)) {
@@ -389,8 +400,8 @@ __global__ void __launch_bounds__(384, 1)
         tmem_st16(tP + part * 16, p);
       }
       if (!ok) break;
-      l += sum;
-      lr += sum_r;
+      l += (sa[0] + sa[1]) + (sa[2] + sa[3]);
+      lr += (sra[0] + sra[1]) + (sra[2] + sra[3]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars->p_full[t]);

@@ -323,6 +323,34 @@ __device__ __forceinline__ float2 unpack2(uint32_t w) {
   return r;
 }
 
+// max(a, b, c) in one instruction (three-operand form of max.f32, sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// acc + (low 16-bit half of w) and acc + (high half), the half widened
+// exactly to fp32 inside the add (mixed-precision add.f32.f16 / .bf16, sm_100).
+template <bool BF16>
+__device__ __forceinline__ float add_lo16(float acc, uint32_t w) {
+  if constexpr (BF16) {
+    asm("{ .reg .b16 lo, hi; mov.b32 {lo, hi}, %1; add.rn.f32.bf16 %0, lo, %0; }" : "+f"(acc) : "r"(w));
+  } else {
+    asm("{ .reg .b16 lo, hi; mov.b32 {lo, hi}, %1; add.rn.f32.f16 %0, lo, %0; }" : "+f"(acc) : "r"(w));
+  }
+  return acc;
+}
+template <bool BF16>
+__device__ __forceinline__ float add_hi16(float acc, uint32_t w) {
+  if constexpr (BF16) {
+    asm("{ .reg .b16 lo, hi; mov.b32 {lo, hi}, %1; add.rn.f32.bf16 %0, hi, %0; }" : "+f"(acc) : "r"(w));
+  } else {
+    asm("{ .reg .b16 lo, hi; mov.b32 {lo, hi}, %1; add.rn.f32.f16 %0, hi, %0; }" : "+f"(acc) : "r"(w));
+  }
+  return acc;
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

@@ -210,30 +210,51 @@ __global__ void __launch_bounds__(384, 1)
           mma_commit(&bars->s_full[1]);
           mma_commit(&bars->kv_empty[0]);
         }
+        // Each half of an iteration first tests its three barriers together:
+        // when this thread runs behind the softmax they have all completed,
+        // and one test replaces three waits in a row.
         for (int j = 0; j < n_kv && ok; ++j) {
           if (j + 1 < n_kv) {
             const int pk = 2 * j + 2;
-            ok = kv_wait(pk);
-            for (int t = 0; t < 2 && ok; ++t) {
-              ok = mbar_wait(&bars->s_cons[t], j & 1, abort);
-              if (!ok) break;
+            if (mbar_ready3(&bars->kv_full[pk % C::kStages], (pk / C::kStages) & 1, &bars->s_cons[0], j & 1,
+                            &bars->s_cons[1], j & 1)) {
               tc_fence_after();
-              issue_s(t, pk % C::kStages);
-              mma_commit(&bars->s_full[t]);
+              issue_s(0, pk % C::kStages);
+              mma_commit(&bars->s_full[0]);
+              issue_s(1, pk % C::kStages);
+              mma_commit(&bars->s_full[1]);
+            } else {
+              ok = kv_wait(pk);
+              for (int t = 0; t < 2 && ok; ++t) {
+                ok = mbar_wait(&bars->s_cons[t], j & 1, abort);
+                if (!ok) break;
+                tc_fence_after();
+                issue_s(t, pk % C::kStages);
+                mma_commit(&bars->s_full[t]);
+              }
+              if (!ok) break;
             }
-            if (!ok) break;
             mma_commit(&bars->kv_empty[pk % C::kStages]);
           }
           const int pv = 2 * j + 1;
-          ok = kv_wait(pv);
-          for (int t = 0; t < 2 && ok; ++t) {
-            ok = mbar_wait(&bars->p_full[t], j & 1, abort);
-            if (!ok) break;
+          if (mbar_ready3(&bars->kv_full[pv % C::kStages], (pv / C::kStages) & 1, &bars->p_full[0], j & 1,
+                          &bars->p_full[1], j & 1)) {
             tc_fence_after();
-            issue_pv(t, pv % C::kStages, j > 0);
-            mma_commit(j + 1 < n_kv ? &bars->pv_done[t] : &bars->o_full[t]);
+            issue_pv(0, pv % C::kStages, j > 0);
+            mma_commit(j + 1 < n_kv ? &bars->pv_done[0] : &bars->o_full[0]);
+            issue_pv(1, pv % C::kStages, j > 0);
+            mma_commit(j + 1 < n_kv ? &bars->pv_done[1] : &bars->o_full[1]);
+          } else {
+            ok = kv_wait(pv);
+            for (int t = 0; t < 2 && ok; ++t) {
+              ok = mbar_wait(&bars->p_full[t], j & 1, abort);
+              if (!ok) break;
+              tc_fence_after();
+              issue_pv(t, pv % C::kStages, j > 0);
+              mma_commit(j + 1 < n_kv ? &bars->pv_done[t] : &bars->o_full[t]);
+            }
+            if (!ok) break;
           }
-          if (!ok) break;
           mma_commit(&bars->kv_empty[pv % C::kStages]);
         }
       } else {

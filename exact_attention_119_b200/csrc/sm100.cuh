@@ -105,6 +105,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Non-blocking test of three phases at once: true when all three have
+// completed. The three tests share one round trip to the barrier unit, where
+// three waits in a row would pay it three times.
+__device__ __forceinline__ bool mbar_ready3(uint64_t* a, uint32_t pa, uint64_t* b, uint32_t pb, uint64_t* c,
+                                            uint32_t pc) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p, q, r;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 q, [%3], %4;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 r, [%5], %6;\n\t"
+      "and.pred p, p, q;\n\t"
+      "and.pred p, p, r;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(a)), "r"(pa), "r"(smem_u32(b)), "r"(pb), "r"(smem_u32(c)), "r"(pc)
+      : "memory");
+  return ok != 0;
+}
+
 // Warp-uniform variant for code that follows with warp-collective tcgen05
 // instructions: every lane returns the same answer.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort) {

@@ -3,6 +3,7 @@
 // caller's stream; nothing here allocates device memory.
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -73,11 +74,36 @@ template <int D, bool CAUSAL, bool BF16>
 cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdArgs& a,
                        cudaStream_t stream) {
   using C = FwdCfg<D>;
-  auto kern = fa_fwd_kernel<D, CAUSAL, BF16>;
+  const unsigned units = static_cast<unsigned>(a.n_mblocks * a.B * a.H);
+  if constexpr (!CAUSAL) {
+    if (a.split == 2) {
+      // Two CTAs per row block, launched as 2-CTA clusters so they are
+      // resident together and can merge through distributed shared memory.
+      auto kern2 = fa_fwd_kernel<D, false, BF16, true>;
+      cudaError_t e = set_smem(kern2, C::kSmemBytes);
+      if (e != cudaSuccess) return e;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * units);
+      cfg.blockDim = dim3(C::kThreads);
+      cfg.dynamicSmemBytes = C::kSmemBytes;
+      cfg.stream = stream;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaLaunchKernelEx(&cfg, kern2, mq, mk, mv, a) == cudaSuccess) return cudaSuccess;
+      (void)cudaGetLastError();  // no cluster fits: run unsplit
+    }
+  }
+  auto kern = fa_fwd_kernel<D, CAUSAL, BF16, false>;
   cudaError_t e = set_smem(kern, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const dim3 grid(a.n_mblocks * a.B * a.H);
-  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, a);
+  FwdArgs one = a;
+  one.split = 1;
+  kern<<<dim3(units), C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, one);
   return cudaGetLastError();
 }
 
@@ -121,6 +147,32 @@ int num_sms() {
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
   return n;
+}
+
+// Forward work split. A row block's key tiles go to one CTA, or are halved
+// between the two CTAs of a cluster when that makes the whole launch shorter.
+// With W CTAs resident at a time, U row blocks of n key tiles take about
+// ceil(U / W) * (n + F) tile-times unsplit and ceil(2U / W) * (ceil(n / 2) + F)
+// + 1 split, where F is a CTA's fixed cost (start, first loads, epilogue) in
+// tile-times and the + 1 is the merge. F = 8 matches a B200 at d = 64: there,
+// 2 x 2048 x 12 heads split (384 CTAs in 3 waves instead of 192 in 2) ran 8%
+// slower. So only launches that leave SMs idle unsplit gain. Causal launches
+// keep one CTA per row block (their longest-first order already fills the
+// machine). FA_FWD_SPLIT=1 or 2 in the environment forces the choice (2 only
+// where a split is possible).
+int fwd_split(int B, int N, int H, bool causal, int n_mblocks) {
+  const int n_kv = (N + 127) / 128;
+  if (causal || n_kv < 2) return 1;
+  if (const char* env = std::getenv("FA_FWD_SPLIT")) {
+    if (env[0] == '1') return 1;
+    if (env[0] == '2') return 2;
+  }
+  constexpr long long kFixed = 8;
+  const long long w = num_sms() > 0 ? num_sms() : 148;
+  const long long units = static_cast<long long>(B) * H * n_mblocks;
+  const long long t1 = (units + w - 1) / w * (n_kv + kFixed);
+  const long long t2 = (2 * units + w - 1) / w * ((n_kv + 1) / 2 + kFixed) + 1;
+  return t2 < t1 ? 2 : 1;
 }
 
 template <int D>
@@ -223,6 +275,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   a.N = N;
   a.H = H;
   a.n_mblocks = (N + 255) / 256;
+  a.split = fwd_split(B, N, H, causal != 0, a.n_mblocks);
   a.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
   const bool bf16 = dtype == FA_BF16;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

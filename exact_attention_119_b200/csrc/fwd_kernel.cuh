@@ -41,6 +41,7 @@ struct FwdArgs {
   float* lse;    // [B, H, N] fp32
   int B, N, H;
   int n_mblocks;       // ceil(N / 256)
+  int split;           // 1, or 2: each row block's key tiles shared by a 2-CTA cluster
   float scale_log2;    // softmax_scale * log2(e)
 };
 
@@ -55,6 +56,9 @@ struct FwdCfg {
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
   static constexpr int kSmemBytes = kBarOff + 512 + 1024;  // + barriers + alignment slack
+  // A split row block's partial state (2 tiles x 128 rows x (D + 4) floats)
+  // goes over Q and the K/V ring at the end.
+  static_assert(2 * 128 * (D + 4) * 4 <= kBarOff, "partial rows must fit below the barriers");
   // TMEM columns: S of tile t at tmem_s(t), O at tmem_o(t), P at tmem_p(t)
   // (its own 64 columns when kSepP, else over S).
   static constexpr bool kSepP = D == 64;
@@ -72,13 +76,14 @@ struct FwdBarriers {
   uint64_t s_cons[2];   // kSepP: the softmax has S(t, j) in registers
   uint64_t pv_done[2];  // kSepP: P(t, j) V_j has completed
   uint64_t drain;
+  uint64_t merge_ready;  // split: the partner's partial rows are in its shared memory
   uint64_t kv_full[8];
   uint64_t kv_empty[8];
   uint32_t tmem_base;
   int abort;
 };
 
-template <int D, bool CAUSAL, bool BF16>
+template <int D, bool CAUSAL, bool BF16, bool SPLIT>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
@@ -92,8 +97,14 @@ __global__ void __launch_bounds__(384, 1)
   const int lane = threadIdx.x & 31;
 
   // Work item: longest-first when causal (the last row block has the most keys).
+  // With split == 2 the two CTAs of a cluster take the first and the second
+  // half of the row block's key tiles, and CTA 0 merges the two partial
+  // results (online-softmax state and unnormalised O) at the end.
   const int bh_count = args.B * args.H;
-  const int item = blockIdx.x;
+  static_assert(!(SPLIT && CAUSAL), "causal launches are not split");
+  constexpr int split = SPLIT ? 2 : 1;
+  const int item = blockIdx.x / split;
+  const uint32_t crank = SPLIT ? cluster_ctarank() : 0u;
   int mblk = item / bh_count;
   const int bh = item % bh_count;
   if (CAUSAL) mblk = args.n_mblocks - 1 - mblk;
@@ -101,7 +112,10 @@ __global__ void __launch_bounds__(384, 1)
   const int h = bh % args.H;
   const int q0 = mblk * 256;
   const int kv_end = CAUSAL ? min(args.N, q0 + 256) : args.N;
-  const int n_kv = (kv_end + C::kKeys - 1) / C::kKeys;
+  const int n_kv_all = (kv_end + C::kKeys - 1) / C::kKeys;
+  const int kv_half = (n_kv_all + 1) / 2;
+  const int kv_lo = crank == 0 ? 0 : kv_half;  // first key tile of this CTA
+  const int n_kv = split == 1 ? n_kv_all : (crank == 0 ? kv_half : n_kv_all - kv_half);
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -113,6 +127,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bars->pv_done[t], 1);
     }
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->merge_ready, 256);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
@@ -127,6 +142,7 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if constexpr (SPLIT) cluster_sync_all();  // partner's barriers initialised before any remote arrive
   const uint32_t tmem = bars->tmem_base;
 
   const uint32_t sQ = smem_u32(smem + C::kQOff);
@@ -159,7 +175,7 @@ __global__ void __launch_bounds__(384, 1)
           const CUtensorMap* map = which == 0 ? &tm_k : &tm_v;
           for (int kb = 0; kb < D / 64; ++kb)
             tma_load_4d(map, smem + C::kKVOff + st * C::kTileBytes + kb * C::kBoxBytes, &bars->kv_full[st],
-                        kb * 64, h, j * C::kKeys, b);
+                        kb * 64, h, (kv_lo + j) * C::kKeys, b);
         }
       }
       // Never leave with copies in flight: wait for the last load on each stage.
@@ -314,7 +330,8 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const uint32_t tS = lane_base + C::tmem_s(t);
     const uint32_t tO = lane_base + C::tmem_o(t);
-    const int lim = CAUSAL ? min(args.N, rg + 1) : args.N;  // keys [0, lim) are kept
+    // Keys [0, lim) are kept; lim is counted from this CTA's first key tile.
+    const int lim = (CAUSAL ? min(args.N, rg + 1) : args.N) - kv_lo * C::kKeys;
     const float c = args.scale_log2;
     // l: sum of the exact p (for LSE); lr: sum of the 16-bit rounded p that
     // P V uses (for O / lr, so each output row's weights add up to one).
@@ -429,29 +446,100 @@ __global__ void __launch_bounds__(384, 1)
     }
 
     // -------------------------------------------------------------- epilogue
-    if (ok && mbar_wait_warp(&bars->o_full[t], 0, abort)) {
-      tc_fence_after();
-      const float inv_l = 1.f / lr;
-      const bool valid = rg < args.N;
-      uint16_t* orow = reinterpret_cast<uint16_t*>(args.o) +
-                       ((static_cast<size_t>(b) * args.N + (valid ? rg : 0)) * args.H + h) * D;
+    if constexpr (!SPLIT) {
+      if (ok && mbar_wait_warp(&bars->o_full[t], 0, abort)) {
+        tc_fence_after();
+        const float inv_l = 1.f / lr;
+        const bool valid = rg < args.N;
+        uint16_t* orow = reinterpret_cast<uint16_t*>(args.o) +
+                         ((static_cast<size_t>(b) * args.N + (valid ? rg : 0)) * args.H + h) * D;
 #pragma unroll 1
-      for (int q = 0; q < D / 32; ++q) {
-        uint32_t o[32];
-        tmem_ld32(tO + q * 32, o);
-        tmem_ld_wait();
-        tie_regs32(o);
-        uint32_t pk[16];
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t o[32];
+          tmem_ld32(tO + q * 32, o);
+          tmem_ld_wait();
+          tie_regs32(o);
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+        if (valid) args.lse[(static_cast<size_t>(b) * args.H + h) * args.N + rg] = m * 0.69314718055994531f + logf(l);
+      }
+    } else {
+      // Split row block. CTA 1 leaves its row state (unnormalised O, m, l,
+      // lr) in its own shared memory, over Q and the K/V ring, which both
+      // tiles' last P V products have finished reading. CTA 0 reads it
+      // through the cluster's shared-memory window and merges: with
+      // M = max(m0, m1) and a_i = 2^(m_i - M), O = (a0 O0 + a1 O1) / (a0 lr0 +
+      // a1 lr1) and l = a0 l0 + a1 l1, the same result as one pass over all
+      // key tiles with running max M. Every softmax thread of CTA 1 arrives on
+      // CTA 0's barrier whatever happened before; neither CTA leaves before
+      // the cluster barrier at the end, after CTA 0's last remote read.
+      const bool done = ok && mbar_wait_warp(&bars->o_full[t], 0, abort) && mbar_wait_warp(&bars->o_full[1 - t], 0, abort);
+      float* part = reinterpret_cast<float*>(smem) + static_cast<size_t>(t * 128 + r) * (D + 4);
+      if (cluster_ctarank() == 1) {
+        if (done) {
+          tc_fence_after();
+#pragma unroll 1
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t o[32];
+            tmem_ld32(tO + q * 32, o);
+            tmem_ld_wait();
+            tie_regs32(o);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              reinterpret_cast<float4*>(part + q * 32)[v] =
+                  make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]), __uint_as_float(o[4 * v + 2]),
+                              __uint_as_float(o[4 * v + 3]));
+          }
+          *reinterpret_cast<float4*>(part + D) = make_float4(m, l, lr, 0.f);
+        }
+        mbar_arrive_remote(mapa_shared(smem_u32(&bars->merge_ready), 0));
+      } else {
+        const bool have = mbar_wait_cluster(&bars->merge_ready, 0);
+        if (done && have) {
+          tc_fence_after();
+          const uint32_t rpart = mapa_shared(smem_u32(part), 1);
+          const float4 st = ld_shared_cluster_v4(rpart + D * 4);  // m1, l1, lr1
+          const float mm = fmaxf(m, st.x);
+          const float a0 = ex2(m - mm), a1 = ex2(st.x - mm);
+          const float l_all = a0 * l + a1 * st.y;
+          const float inv = 1.f / (a0 * lr + a1 * st.z);
+          const float c0 = a0 * inv, c1 = a1 * inv;
+          const bool valid = rg < args.N;
+          uint16_t* orow = reinterpret_cast<uint16_t*>(args.o) +
+                           ((static_cast<size_t>(b) * args.N + (valid ? rg : 0)) * args.H + h) * D;
+#pragma unroll 1
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t o[32];
+            tmem_ld32(tO + q * 32, o);
+            tmem_ld_wait();
+            tie_regs32(o);
+            uint32_t pk[16];
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const float4 x = ld_shared_cluster_v4(rpart + (q * 32 + 4 * v) * 4);
+              pk[2 * v] = pack2<BF16>(fmaf(__uint_as_float(o[4 * v]), c0, x.x * c1),
+                                      fmaf(__uint_as_float(o[4 * v + 1]), c0, x.y * c1));
+              pk[2 * v + 1] = pack2<BF16>(fmaf(__uint_as_float(o[4 * v + 2]), c0, x.z * c1),
+                                          fmaf(__uint_as_float(o[4 * v + 3]), c0, x.w * c1));
+            }
+            if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+#pragma unroll
+              for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
+          }
+          if (valid)
+            args.lse[(static_cast<size_t>(b) * args.H + h) * args.N + rg] = mm * 0.69314718055994531f + logf(l_all);
         }
       }
-      if (valid) args.lse[(static_cast<size_t>(b) * args.H + h) * args.N + rg] = m * 0.69314718055994531f + logf(l);
     }
   } else {
     reg_alloc_dec<104>();  // warps 10-11: no role
@@ -463,6 +551,9 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  // Every thread of both CTAs gets here after bounded waits only; no CTA of a
+  // split pair leaves while the other may still touch its shared memory.
+  if constexpr (SPLIT) cluster_sync_all();
 }
 
 }  // namespace fa

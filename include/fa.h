@@ -77,6 +77,13 @@ typedef enum { FA_FP16 = 0, FA_BF16 = 1 } fa_dtype;
  *   lse      out: [B, H, N] fp32, natural-log logsumexp of the scaled
  *                 (and masked) logits of each query row; fa_bwd needs it.
  *   causal   0 = full attention; 1 = query i attends keys 0..i.
+ * Work split: where it shortens the launch (few row blocks per SM), a
+ * non-causal call halves each row block's key tiles between the two CTAs of
+ * a 2-CTA cluster, and one merges the two online-softmax states (rescale by
+ * the larger running max, add O and l) before O and lse are written. The
+ * choice follows the shape and the device's SM count; FA_FWD_SPLIT=1 or 2 in
+ * the environment forces it. The two paths round differently, each
+ * deterministically.
  */
 FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N, int H, int d,
                  float softmax_scale, int causal, fa_dtype dtype, fa_stream_t stream);

@@ -124,3 +124,21 @@ def test_outputs_not_written_past_n():
     torch.cuda.synchronize()
     assert torch.all(big[130 * 2 * 64:] == 7.0)
     assert torch.all(lse_big[2 * 130:] == 9.0)
+
+
+@pytest.mark.parametrize("split", ["1", "2"])
+@pytest.mark.parametrize("N", [129, 300, 1000, 2048])
+@pytest.mark.parametrize("d,dtype", [(64, "fp16"), (128, "bf16")])
+def test_forced_key_split(monkeypatch, split, N, d, dtype):
+    # Both work splits agree with the oracle: one CTA per row block, and a
+    # 2-CTA cluster that halves the key tiles (odd counts included) and merges
+    # the two online-softmax states.
+    monkeypatch.setenv("FA_FWD_SPLIT", split)
+    check_full(Case(1, N, 2, d, dtype, False, seed=N + int(split)))
+
+
+@pytest.mark.parametrize("split", ["1", "2"])
+def test_forced_key_split_large_logits(monkeypatch, split):
+    # The two halves see very different row maxima; the merge rescales by them.
+    monkeypatch.setenv("FA_FWD_SPLIT", split)
+    check_full(Case(1, 2048, 4, 128, "bf16", False, sigma_qk=3.0, seed=5))

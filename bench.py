@@ -50,8 +50,8 @@ DEFAULT_WORKLOAD = "p4_B2_N2048_H12_d64_fp16"
 # ncu DRAM bytes per launch of the dominant kernel, from the capture summarised
 # in profiles/ for the default workload; None when the kernel has changed since.
 NCU_TRAFFIC_BYTES = {
-    # fa_bwd_dkdv<64,0,0>: dram__bytes_read.sum 25,630,720 + dram__bytes_write.sum 345,856
-    ("p4_B2_N2048_H12_d64_fp16", "fa_bwd_dkdv"): 25_976_576,
+    # fa_bwd_dkdv<64,0,0>: dram__bytes_read.sum 25,630,976 + dram__bytes_write.sum 304,384
+    ("p4_B2_N2048_H12_d64_fp16", "fa_bwd_dkdv"): 25_935_360,
 }
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}

@@ -24,6 +24,11 @@
 // exponential unit is not left idle waiting for the next S. At d = 128 P
 // overwrites S in place and the next S follows P V.
 //
+// Split (SPLIT = true, non-causal launches that would leave SMs idle): the two
+// CTAs of a 2-CTA cluster take the first and second half of a row block's key
+// tiles, and CTA 0 merges CTA 1's online-softmax state (unnormalised O, m, l)
+// through the cluster's shared-memory window before writing O and LSE.
+//
 // Online softmax with a lagging reference max: the running max m (log2
 // units) is only moved, and O and l rescaled, when a tile's max exceeds m by
 // more than kRescaleLog2 (so P <= 2^kRescaleLog2). The final O / l and

@@ -62,6 +62,16 @@ def flops(B, N, H, d, causal):
     return 4 * base, 10 * base
 
 
+def exp_rate(B, N, H, causal, ms_sum, steps, world, sm_mhz, n_sm):
+    """Exponentials per second in one pass (the forward, or the backward's
+    recompute of P: one exp per unmasked score, halved when causal), whole job,
+    and the exp unit's rate at the sampled SM clock (16 per clock per SM)."""
+    count = B * H * N * N * (0.5 if causal else 1.0)
+    achieved = world * steps * count / (ms_sum * 1e-3)
+    peak = 16.0 * n_sm * sm_mhz * 1e6 * world if sm_mhz else None
+    return achieved, peak
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -412,6 +422,17 @@ def main():
             "gpu_launches": 4 * args.steps,
             "clocks": clocks,
         }
+        try:
+            sm_mhz = (clocks or {}).get("sm_mhz")
+            n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+            ef, peak_e = exp_rate(B, N, H, causal, fwd_sum, args.steps, world, sm_mhz, n_sm)
+            eb, _ = exp_rate(B, N, H, causal, bwd_sum, args.steps, world, sm_mhz, n_sm)
+            line["exp_throughput"] = {
+                "fwd_per_s": ef, "bwd_per_s": eb, "peak_per_s": peak_e,
+                "fwd_frac": ef / peak_e if peak_e else None, "bwd_frac": eb / peak_e if peak_e else None,
+                "note": "one exp per unmasked score per pass; peak = 16/clk/SM x SMs x median sampled SM clock"}
+        except Exception as exc:  # a secondary figure; never lose the bench line over it
+            line["exp_throughput"] = {"error": str(exc)[:200]}
         if extra:
             for v in extra.values():
                 v["fwd_frac_of_peak"] = v["fwd_tflops"] / peak

@@ -50,3 +50,16 @@ def test_flops_counting():
 def test_single_rank_is_identity():
     import bench
     assert bench.reduce_max([1.0, 2.0], 1) == [1.0, 2.0]
+
+
+def test_exp_rate_counts_one_exp_per_unmasked_score():
+    import bench
+    # 2 x 8 heads x 1024^2 scores, 10 steps in 5 ms on one GPU at 1000 MHz on 100 SMs
+    got, peak = bench.exp_rate(2, 1024, 8, False, 5.0, 10, 1, 1000.0, 100)
+    assert got == 2 * 8 * 1024 * 1024 * 10 / 5e-3
+    assert peak == 16 * 100 * 1000e6
+    half, _ = bench.exp_rate(2, 1024, 8, True, 5.0, 10, 1, 1000.0, 100)
+    assert half == got / 2
+    two, peak2 = bench.exp_rate(2, 1024, 8, False, 5.0, 10, 2, 1000.0, 100)
+    assert two == 2 * got and peak2 == 2 * peak
+    assert bench.exp_rate(1, 1, 1, False, 1.0, 1, 1, None, 148)[1] is None

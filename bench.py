@@ -423,7 +423,8 @@ def main():
             "clocks": clocks,
         }
         try:
-            sm_mhz = (clocks or {}).get("sm_mhz")
+            # median sampled SM clock; the maximum clock when no sample fell inside the window
+            sm_mhz = (clocks or {}).get("sm_mhz") or (clocks or {}).get("sm_max_mhz")
             n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
             ef, peak_e = exp_rate(B, N, H, causal, fwd_sum, args.steps, world, sm_mhz, n_sm)
             eb, _ = exp_rate(B, N, H, causal, bwd_sum, args.steps, world, sm_mhz, n_sm)

@@ -129,3 +129,21 @@ def test_workspace_reuse_and_no_overrun():
         assert torch.equal(x, y)
     for b in bufs:
         assert torch.all(b[n:] == 3.0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_autograd_wrapper_matches_direct_calls(causal):
+    # flash_attn_func (torch.autograd.Function over fa_fwd / fa_bwd) returns
+    # exactly what the direct calls return; the backward is deterministic.
+    import exact_attention_119_b200 as fa
+    case = Case(1, 300, 2, 64, "fp16", causal, seed=3)
+    q, k, v, do = (case.torch(n) for n in ("q", "k", "v", "do"))
+    qr, kr, vr = (t.clone().requires_grad_(True) for t in (q, k, v))
+    y = fa.flash_attn_func(qr, kr, vr, case.scale, causal)
+    y.backward(do)
+    o, lse = fa.forward(q, k, v, case.scale, causal)
+    dq, dk, dv = fa.backward(q, k, v, o, do, lse, case.scale, causal)
+    torch.cuda.synchronize()
+    assert torch.equal(y.detach(), o)
+    for got, want in ((qr.grad, dq), (kr.grad, dk), (vr.grad, dv)):
+        assert torch.equal(got, want)

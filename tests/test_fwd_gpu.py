@@ -142,3 +142,17 @@ def test_forced_key_split_large_logits(monkeypatch, split):
     # The two halves see very different row maxima; the merge rescales by them.
     monkeypatch.setenv("FA_FWD_SPLIT", split)
     check_full(Case(1, 2048, 4, 128, "bf16", False, sigma_qk=3.0, seed=5))
+
+
+def test_forced_split_leaves_causal_unsplit(monkeypatch):
+    # Causal launches are never split; forcing the split must not change them.
+    import exact_attention_119_b200 as fa
+    case = Case(1, 1000, 2, 64, "fp16", True, seed=11)
+    q, k, v = case.torch("q"), case.torch("k"), case.torch("v")
+    monkeypatch.setenv("FA_FWD_SPLIT", "1")
+    o1, l1 = fa.forward(q, k, v, case.scale, True)
+    monkeypatch.setenv("FA_FWD_SPLIT", "2")
+    o2, l2 = fa.forward(q, k, v, case.scale, True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    check_full(case)

@@ -259,13 +259,14 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
 // query tile i it adds into the lower sum (chain 0) when i >= j and into the
 // upper sum (chain 1) when i < j; pos(i) is its place in that chain's order
 // (0 = first, which stores instead of adding).
+// (Host-callable too, so the schedule's properties are checked on the CPU.)
 struct BwdItem {
   int bh, j, T, n;
-  __device__ __forceinline__ int tile(int s) const { return j + s < n ? j + s : j + s - n; }
-  __device__ __forceinline__ int chain(int i) const { return i >= j ? 0 : 1; }
-  __device__ __forceinline__ int pos(int i) const { return i >= j ? i - j : n - 1 - j; }
+  __host__ __device__ __forceinline__ int tile(int s) const { return j + s < n ? j + s : j + s - n; }
+  __host__ __device__ __forceinline__ int chain(int i) const { return i >= j ? 0 : 1; }
+  __host__ __device__ __forceinline__ int pos(int i) const { return i >= j ? i - j : n - 1 - j; }
 };
-__device__ __forceinline__ BwdItem decode_item(int item, int ntiles, bool causal) {
+__host__ __device__ __forceinline__ BwdItem decode_item(int item, int ntiles, bool causal) {
   BwdItem it;
   it.bh = item / ntiles;
   it.j = ntiles - 1 - item % ntiles;  // descending j within a head

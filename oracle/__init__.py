@@ -4,7 +4,9 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package; the CUDA path never does.
 """
 
-from .attention import (attention_backward, attention_forward, default_scale,
+from .attention import (attention_backward, attention_backward_varlen, attention_forward,
+                        attention_forward_kvcache, attention_forward_varlen, default_scale,
                         online_softmax_forward)
 
-__all__ = ["attention_forward", "attention_backward", "online_softmax_forward", "default_scale"]
+__all__ = ["attention_forward", "attention_backward", "online_softmax_forward", "default_scale",
+           "attention_forward_varlen", "attention_backward_varlen", "attention_forward_kvcache"]

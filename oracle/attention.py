@@ -99,6 +99,17 @@ def attention_forward(q, k, v, scale: float, causal: bool = False, rows=None):
     return o, lse
 
 
+def _head_backward(qh, kh, vh, doh, scale: float, causal: bool):
+    """dQ, dK, dV and D of one head (textbook chain rule through softmax)."""
+    rows = np.arange(qh.shape[0])
+    p, _ = _softmax_rows(_scores(qh, kh, scale, rows, causal))
+    dvh = p.T @ doh
+    dp = doh @ vh.T
+    drow = (p * dp).sum(axis=1)
+    ds = p * (dp - drow[:, None])
+    return scale * (ds @ kh), scale * (ds.T @ qh), dvh, drow
+
+
 def attention_backward(q, k, v, do, scale: float, causal: bool = False, heads=None):
     """Gradients (dQ, dK, dV) of L = sum(dO o O) for the attention above, fp64.
 
@@ -113,18 +124,9 @@ def attention_backward(q, k, v, do, scale: float, causal: bool = False, heads=No
     dv = np.full_like(q, np.nan)
     dd = np.full((B, H, N), np.nan)
     pairs = [(b, h) for b in range(B) for h in range(H)] if heads is None else list(heads)
-    rows = np.arange(N)
     for b, h in pairs:
-        qh, kh, vh, doh = q[b, :, h, :], k[b, :, h, :], v[b, :, h, :], do[b, :, h, :]
-        p, _ = _softmax_rows(_scores(qh, kh, scale, rows, causal))
-        dvh = p.T @ doh
-        dp = doh @ vh.T
-        drow = (p * dp).sum(axis=1)
-        ds = p * (dp - drow[:, None])
-        dq[b, :, h, :] = scale * (ds @ kh)
-        dk[b, :, h, :] = scale * (ds.T @ qh)
-        dv[b, :, h, :] = dvh
-        dd[b, h, :] = drow
+        dq[b, :, h, :], dk[b, :, h, :], dv[b, :, h, :], dd[b, h, :] = _head_backward(
+            q[b, :, h, :], k[b, :, h, :], v[b, :, h, :], do[b, :, h, :], scale, causal)
     return dq, dk, dv, dd
 
 
@@ -173,3 +175,96 @@ def online_softmax_forward(q, k, v, scale: float, causal: bool, tile_sizes):
 def default_scale(d: int) -> float:
     """softmax_scale=None means 1/sqrt(head_dim) ([P3] §4.2 and §6.2)."""
     return 1.0 / math.sqrt(d)
+
+
+# ------------------------------------------------------------ variable length
+
+def _as_packed(x) -> np.ndarray:
+    a = np.asarray(x, dtype=np.float64)
+    if a.ndim != 3:
+        raise ValueError("expected a packed [total, heads, head_dim] array")
+    return a
+
+
+def _seq_bounds(cu_seqlens, total: int):
+    cu = [int(c) for c in cu_seqlens]
+    if cu[0] != 0 or cu[-1] != total or any(b < a for a, b in zip(cu, cu[1:])):
+        raise ValueError("cu_seqlens must start at 0, not decrease and end at total")
+    return list(zip(cu[:-1], cu[1:]))
+
+
+def attention_forward_varlen(q, k, v, cu_seqlens, scale: float, causal: bool = False):
+    """Variable-length batch, packed without padding ([P3] §4.2, third pitfall:
+    variable-length sequences go through flash_attn_varlen_func).
+
+    q, k, v: [total, H, d]; sequence b owns rows cu_seqlens[b] ..
+    cu_seqlens[b+1] - 1 of all three and attends only to itself (causal: key
+    j of the sequence for query i of the sequence iff j <= i). Each sequence is
+    the plain definition on its own rows. Returns O [total, H, d] and
+    LSE [H, total] (row r of the packed tensors at column r).
+    """
+    q, k, v = _as_packed(q), _as_packed(k), _as_packed(v)
+    total, H, d = q.shape
+    o = np.full((total, H, d), np.nan)
+    lse = np.full((H, total), np.nan)
+    for a, e in _seq_bounds(cu_seqlens, total):
+        if e == a:
+            continue
+        rows = np.arange(e - a)
+        for h in range(H):
+            p, lse_rows = _softmax_rows(_scores(q[a:e, h], k[a:e, h], scale, rows, causal))
+            o[a:e, h] = p @ v[a:e, h]
+            lse[h, a:e] = lse_rows
+    return o, lse
+
+
+def attention_backward_varlen(q, k, v, do, cu_seqlens, scale: float, causal: bool = False):
+    """Gradients of the variable-length forward above: each sequence's dQ, dK,
+    dV and D by the chain rule on its own rows. Returns dQ, dK, dV
+    [total, H, d] and D [H, total]."""
+    q, k, v, do = _as_packed(q), _as_packed(k), _as_packed(v), _as_packed(do)
+    total, H, d = q.shape
+    dq, dk, dv = (np.full((total, H, d), np.nan) for _ in range(3))
+    dd = np.full((H, total), np.nan)
+    for a, e in _seq_bounds(cu_seqlens, total):
+        if e == a:
+            continue
+        for h in range(H):
+            dq[a:e, h], dk[a:e, h], dv[a:e, h], dd[h, a:e] = _head_backward(
+                q[a:e, h], k[a:e, h], v[a:e, h], do[a:e, h], scale, causal)
+    return dq, dk, dv, dd
+
+
+# ----------------------------------------------------------- KV-cache decode
+
+def attention_forward_kvcache(q, k_cache, v_cache, cache_seqlens, scale: float, causal: bool = False):
+    """Decode step against a key/value cache ([P3] §6.1: inference with a KV
+    cache whose length grows one step at a time).
+
+    q: [B, Nq, H, d], the Nq newest positions of each sequence; k_cache,
+    v_cache: [B, Nmax, H, d], of which batch b holds L_b = cache_seqlens[b]
+    valid rows (the Nq newest included). Query t of batch b sits at position
+    L_b - Nq + t; it attends keys 0 .. L_b - 1, or with ``causal`` keys
+    0 .. L_b - Nq + t (its own position and earlier). A query with no key to
+    attend (L_b - Nq + t < 0 under ``causal``, or L_b = 0) gets O = 0 and
+    LSE = -inf. Returns O [B, Nq, H, d] and LSE [B, H, Nq].
+    """
+    q, kc, vc = _as_f64(q), _as_f64(k_cache), _as_f64(v_cache)
+    B, Nq, H, d = q.shape
+    o = np.zeros((B, Nq, H, d))
+    lse = np.full((B, H, Nq), -np.inf)
+    for b in range(B):
+        L = int(cache_seqlens[b])
+        if not 0 <= L <= kc.shape[1]:
+            raise ValueError("cache length out of range")
+        for t in range(Nq):
+            last = L - 1 if not causal else L - Nq + t
+            if last < 0:
+                continue
+            for h in range(H):
+                s = scale * (kc[b, :last + 1, h] @ q[b, t, h])
+                m = s.max()
+                e = np.exp(s - m)
+                o[b, t, h] = (e @ vc[b, :last + 1, h]) / e.sum()
+                lse[b, h, t] = m + np.log(e.sum())
+    return o, lse

@@ -268,3 +268,76 @@ def attention_forward_kvcache(q, k_cache, v_cache, cache_seqlens, scale: float, 
                 o[b, t, h] = (e @ vc[b, :last + 1, h]) / e.sum()
                 lse[b, h, t] = m + np.log(e.sum())
     return o, lse
+
+
+# ------------------------------------------------------------------ dropout
+
+def dropout_threshold(p: float) -> int:
+    """The integer form of a dropout probability: an element is dropped when
+    its 32-bit random word is below floor(p * 2^32) (so p = 0 drops nothing).
+    Both sides receive this integer; no floating point decides a mask bit."""
+    if not 0.0 <= p < 1.0:
+        raise ValueError("dropout probability must be in [0, 1)")
+    return min(int(p * 4294967296.0), 4294967295)
+
+
+def dropout_keep(b: int, h: int, H: int, nq: int, nk: int, p: float, seed: int, offset: int) -> np.ndarray:
+    """Keep mask [nq, nk] of head (b, h) (b: the sequence when variable-length).
+
+    The dropout of P ([P2] usage line and [P3] §4.2: flash_attn_func takes
+    dropout_p) needs a mask that the backward pass can regenerate instead of
+    storing; the pages give no generator, so this one is Philox4x32-10 (see
+    oracle/philox.py) with key (seed mod 2^32, seed >> 32) and counter
+    (j // 4, i, b*H + h, offset) for query i and key j of the sequence; word
+    j % 4 of that call is element (i, j)'s draw.
+    """
+    from .philox import philox4x32_10
+    i = np.arange(nq, dtype=np.uint64)[:, None]
+    j = np.arange(nk, dtype=np.uint64)[None, :]
+    words = philox4x32_10(j >> np.uint64(2), i, np.uint64(b * H + h), np.uint64(offset),
+                          np.uint64(seed & 0xFFFFFFFF), np.uint64((seed >> 32) & 0xFFFFFFFF))
+    w = np.choose((j & np.uint64(3)).astype(np.int64) + np.zeros((nq, 1), dtype=np.int64), words)
+    return w >= np.uint32(dropout_threshold(p))
+
+
+def attention_forward_dropout(q, k, v, scale: float, causal: bool, p: float, seed: int, offset: int = 0):
+    """O = (P o Z) V with Z = keep / (1 - p) elementwise (inverted dropout on
+    the attention probabilities), and the LSE of the undropped softmax, fp64.
+    The keep mask is dropout_keep()'s."""
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, N, H, d = q.shape
+    o = np.empty((B, N, H, d))
+    lse = np.empty((B, H, N))
+    rows = np.arange(N)
+    for b in range(B):
+        for h in range(H):
+            pr, lse_rows = _softmax_rows(_scores(q[b, :, h], k[b, :, h], scale, rows, causal))
+            z = dropout_keep(b, h, H, N, N, p, seed, offset) / (1.0 - p)
+            o[b, :, h] = (pr * z) @ v[b, :, h]
+            lse[b, h] = lse_rows
+    return o, lse
+
+
+def attention_backward_dropout(q, k, v, do, scale: float, causal: bool, p: float, seed: int, offset: int = 0):
+    """Gradients of attention_forward_dropout (the mask does not depend on the
+    inputs): dV = (P o Z)^T dO, dP = (dO V^T) o Z, D_i = sum_j P_ij dP_ij
+    (= rowsum(dO o O)), dS = P o (dP - D), dQ = scale dS K, dK = scale dS^T Q.
+    Returns dQ, dK, dV [B, N, H, d] and D [B, H, N]."""
+    q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
+    B, N, H, d = q.shape
+    dq, dk, dv = (np.empty((B, N, H, d)) for _ in range(3))
+    dd = np.empty((B, H, N))
+    rows = np.arange(N)
+    for b in range(B):
+        for h in range(H):
+            qh, kh, vh, doh = q[b, :, h], k[b, :, h], v[b, :, h], do[b, :, h]
+            pr, _ = _softmax_rows(_scores(qh, kh, scale, rows, causal))
+            z = dropout_keep(b, h, H, N, N, p, seed, offset) / (1.0 - p)
+            dv[b, :, h] = (pr * z).T @ doh
+            dp = (doh @ vh.T) * z
+            drow = (pr * dp).sum(axis=1)
+            ds = pr * (dp - drow[:, None])
+            dq[b, :, h] = scale * (ds @ kh)
+            dk[b, :, h] = scale * (ds.T @ qh)
+            dd[b, h] = drow
+    return dq, dk, dv, dd

@@ -193,7 +193,7 @@ def _seq_bounds(cu_seqlens, total: int):
     return list(zip(cu[:-1], cu[1:]))
 
 
-def attention_forward_varlen(q, k, v, cu_seqlens, scale: float, causal: bool = False):
+def attention_forward_varlen(q, k, v, cu_seqlens, scale: float, causal: bool = False, dropout=None):
     """Variable-length batch, packed without padding ([P3] §4.2, third pitfall:
     variable-length sequences go through flash_attn_varlen_func).
 
@@ -201,18 +201,25 @@ def attention_forward_varlen(q, k, v, cu_seqlens, scale: float, causal: bool = F
     cu_seqlens[b+1] - 1 of all three and attends only to itself (causal: key
     j of the sequence for query i of the sequence iff j <= i). Each sequence is
     the plain definition on its own rows. Returns O [total, H, d] and
-    LSE [H, total] (row r of the packed tensors at column r).
+    LSE [H, total] (row r of the packed tensors at column r). ``dropout``:
+    optional (p, seed, offset), the mask of dropout_keep() with b the
+    sequence's index and i, j counted from its first row.
     """
     q, k, v = _as_packed(q), _as_packed(k), _as_packed(v)
     total, H, d = q.shape
     o = np.full((total, H, d), np.nan)
     lse = np.full((H, total), np.nan)
-    for a, e in _seq_bounds(cu_seqlens, total):
+    bounds = _seq_bounds(cu_seqlens, total)
+    seq_index = {ae: b for b, ae in enumerate(bounds)}
+    for a, e in bounds:
         if e == a:
             continue
         rows = np.arange(e - a)
         for h in range(H):
             p, lse_rows = _softmax_rows(_scores(q[a:e, h], k[a:e, h], scale, rows, causal))
+            if dropout is not None:
+                pd, seed, offset = dropout
+                p = p * dropout_keep(seq_index[a, e], h, H, e - a, e - a, pd, seed, offset) / (1.0 - pd)
             o[a:e, h] = p @ v[a:e, h]
             lse[h, a:e] = lse_rows
     return o, lse

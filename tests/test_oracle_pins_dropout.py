@@ -99,3 +99,20 @@ def test_dropout_gradients_match_finite_differences(causal):
     # D = rowsum(dO o O) holds with dropout too
     o, _ = attention_forward_dropout(q, k, v, 0.7, causal, p, seed)
     np.testing.assert_allclose(dd, (do * o).sum(axis=3).transpose(0, 2, 1), atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_dropout_equals_fixed_length_batch(causal):
+    # Equal-length sequences packed with cu_seqlens are the fixed-length batch,
+    # dropout mask included (sequence b draws with b*H + h, i and j counted
+    # from its first row).
+    from oracle import attention_forward_varlen
+    rng = np.random.default_rng(12)
+    B, N, H, d = 3, 10, 2, 4
+    q, k, v = (rng.standard_normal((B, N, H, d)) for _ in range(3))
+    o, lse = attention_forward_dropout(q, k, v, 0.5, causal, 0.3, seed=77, offset=5)
+    cu = np.arange(B + 1) * N
+    ov, lv = attention_forward_varlen(q.reshape(B * N, H, d), k.reshape(B * N, H, d), v.reshape(B * N, H, d), cu,
+                                      0.5, causal, dropout=(0.3, 77, 5))
+    np.testing.assert_allclose(ov, o.reshape(B * N, H, d), atol=1e-13)
+    np.testing.assert_allclose(lv, lse.transpose(1, 0, 2).reshape(H, B * N), atol=1e-13)

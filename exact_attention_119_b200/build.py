@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfa.so")
 SOURCES = ["fa_api.cu"]
-HEADERS = ["sm100.cuh", "fwd_kernel.cuh", "bwd_kernels.cuh"]
+HEADERS = ["sm100.cuh", "fwd_kernel.cuh", "bwd_kernels.cuh", "decode_kernels.cuh"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 

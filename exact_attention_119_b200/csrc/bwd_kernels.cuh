@@ -21,16 +21,13 @@
 //                    added into fp32 accumulators in a fixed key-tile order
 //                    (per-tile counters say whose turn it is), so the sum is
 //                    deterministic.
-//   3. fa_bwd_dq:    dQ = scale * (lower + upper accumulator), cast.
+//   3. fa_bwd_dq:    dQ = scale * (lower sum + upper sum), cast.
 //
-// dQ order. Key tile j visits query tiles i = j, j+1, ..., n-1 and then (non-
-// causal only) 0, 1, ..., j-1. Query tile i collects two sums: the lower one
-// from j = i, i-1, ..., 0 and the upper one from j = n-1, n-2, ..., i+1, each
-// in descending j. Items are handed out in descending j within a head, so the
-// contributor a tile waits for (j+1) was fetched earlier, and in steady state
-// it visited that tile one step earlier: the wait is already over. No wait can
-// deadlock (the earliest-fetched unfinished item waits for nothing), and
-// every wait is bounded anyway.
+// dQ order (BwdItem below). Query tile i's dQ is summed in fp32 over key
+// tiles in a fixed descending order (two sums when non-causal, added in a
+// fixed order at the end), so the result does not depend on scheduling. No
+// wait can deadlock (the earliest-fetched unfinished item waits for nothing),
+// and every wait is bounded anyway.
 #pragma once
 
 #include <algorithm>
@@ -62,18 +59,32 @@ struct BwdLayout {
 };
 
 struct BwdArgs {
+  // Caller tensors: element (b, n, h, c) of X at X[b*X_sb + (row0 + n)*X_sn +
+  // h*X_sh + c] (row0 = 0, or the sequence's first row when variable-length).
   const uint16_t* o;
+  long long o_sb, o_sn, o_sh;
   const uint16_t* dout;
-  const float* lse;
+  long long do_sb, do_sn, do_sh;
+  const float* lse;  // at lse[b*lse_sb + h*lse_sh + row0 + n]
+  long long lse_sb, lse_sh;
   uint16_t* dq;
+  long long dq_sb, dq_sn, dq_sh;
   uint16_t* dk;
+  long long dk_sb, dk_sn, dk_sh;
   uint16_t* dv;
-  float* lse2;   // [B*H, npad] LSE * log2(e); +inf on pad rows
-  float* dd;     // [B*H, npad] D; 0 on pad rows
+  long long dv_sb, dv_sn, dv_sh;
+  const int* cu;     // variable-length row offsets [B + 1], or nullptr
+  int total;         // rows of the packed tensors (variable length)
+  // Workspace
+  float* lse2;   // [B*H, npad] LSE * log2(e); +inf on rows past the sequence
+  float* dd;     // [B*H, npad] D; 0 on rows past the sequence
   float* dqacc;  // 2 x [B*H, ntiles, d/4, 128, 4] fp32 (lower, upper sums)
   int* cnt;      // 2 x [B*H, ntiles] dQ ordering counters (lower, upper)
   int* sched;    // work counter
-  int B, N, H, npad, ntiles;
+  int B, N, H, npad, ntiles;  // N: sequence length (variable length: the longest)
+  int d;             // head size (<= D; columns d .. D-1 are zeros from TMA)
+  uint32_t hm;       // head-major tensor maps (kHmQ | kHmK | kHmV | kHmDO)
+  Dropout drop;      // used by the DROPOUT instantiation only
   float scale;       // softmax_scale
   float scale_log2;  // softmax_scale * log2(e)
 };
@@ -82,22 +93,29 @@ struct BwdArgs {
 
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256) fa_bwd_prep(const BwdArgs a) {
-  // A group of G = D/8 lanes per (b, n, h) row, 8 elements per lane; the
-  // warp's groups take consecutive rows so the loop stays warp-uniform.
+  // A group of G = D/8 lanes per (b, h, n) row, 8 elements per lane, over
+  // n < npad of every head: rows of the sequence get D = rowsum(dO o O) and
+  // LSE*log2(e); rows past its end get 0 and +inf (no query: P = 0).
   constexpr int G = D / 8;
   const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   const long long nthreads = (long long)gridDim.x * blockDim.x;
-  const long long rows = (long long)a.B * a.N * a.H;
+  const long long rows = (long long)a.B * a.H * a.npad;
   const int lane = threadIdx.x & 31;
   const int sub = lane % G;
   const long long ngroups = nthreads / G;
   for (long long row0 = (tid / 32) * (32 / G); row0 < rows; row0 += ngroups) {
-    const long long row = row0 + lane / G;
-    const bool valid = row < rows;
+    const long long row = row0 + lane / G;  // bh * npad + n
+    const bool in = row < rows;
+    const int bh = in ? (int)(row / a.npad) : 0;
+    const int n = in ? (int)(row % a.npad) : 0;
+    const int b = bh / a.H, h = bh % a.H;
+    const SeqRows seq = seq_rows(a.cu, b, a.N, a.total);
+    const bool valid = in && n < seq.len;
     float acc = 0.f;
-    if (valid) {
-      const uint4 ov = reinterpret_cast<const uint4*>(a.o + row * D)[sub];
-      const uint4 dv = reinterpret_cast<const uint4*>(a.dout + row * D)[sub];
+    if (valid && sub * 8 < a.d) {
+      const long long r = seq.row0 + n;
+      const uint4 ov = *reinterpret_cast<const uint4*>(a.o + b * a.o_sb + r * a.o_sn + h * a.o_sh + sub * 8);
+      const uint4 dv = *reinterpret_cast<const uint4*>(a.dout + b * a.do_sb + r * a.do_sn + h * a.do_sh + sub * 8);
       const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
       const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
 #pragma unroll
@@ -110,24 +128,10 @@ __global__ void __launch_bounds__(256) fa_bwd_prep(const BwdArgs a) {
     }
 #pragma unroll
     for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, G);
-    if (valid && sub == 0) {
-      const int h = (int)(row % a.H);
-      const long long bn = row / a.H;
-      const int n = (int)(bn % a.N);
-      const int b = (int)(bn / a.N);
-      const size_t idx = ((size_t)b * a.H + h) * a.npad + n;
-      a.dd[idx] = acc;
-      a.lse2[idx] = a.lse[((size_t)b * a.H + h) * a.N + n] * 1.4426950408889634f;
+    if (in && sub == 0) {
+      a.dd[row] = valid ? acc : 0.f;
+      a.lse2[row] = valid ? a.lse[b * a.lse_sb + h * a.lse_sh + seq.row0 + n] * 1.4426950408889634f : INFINITY;
     }
-  }
-  // Pad rows (no query there: P = 0 through LSE = +inf), counters, work counter.
-  const int padn = a.npad - a.N;
-  const long long pads = (long long)a.B * a.H * padn;
-  for (long long p = tid; p < pads; p += nthreads) {
-    const long long bh = p / padn;
-    const int n = a.N + (int)(p % padn);
-    a.dd[bh * a.npad + n] = 0.f;
-    a.lse2[bh * a.npad + n] = INFINITY;
   }
   const long long ncnt = 2LL * a.B * a.H * a.ntiles;
   for (long long p = tid; p < ncnt; p += nthreads) a.cnt[p] = 0;
@@ -148,20 +152,22 @@ __global__ void __launch_bounds__(256) fa_bwd_dq(const BwdArgs a) {
     const int c4 = (int)(rest % (D / 4));
     rest /= (D / 4);
     const int tile = (int)(rest % a.ntiles);
-    const long long bh = rest / a.ntiles;
+    const int bh = (int)(rest / a.ntiles);
     const int n = tile * 128 + r;
-    if (n >= a.N) continue;
+    const int b = bh / a.H, h = bh % a.H;
+    const SeqRows seq = seq_rows(a.cu, b, a.N, a.total);
+    if (n >= seq.len || c4 * 4 >= a.d) continue;
     float4 v = reinterpret_cast<const float4*>(a.dqacc)[t];
-    if (!CAUSAL && tile < a.ntiles - 1) {
-      // Upper sum (key tiles after this query tile): present unless i = n-1.
+    if (!CAUSAL && tile < (seq.len + 127) / 128 - 1) {
+      // Upper sum (key tiles after this query tile): present unless i is the
+      // sequence's last tile.
       const float4 u = reinterpret_cast<const float4*>(a.dqacc)[t + total];
       v.x += u.x;
       v.y += u.y;
       v.z += u.z;
       v.w += u.w;
     }
-    const int b = (int)(bh / a.H), h = (int)(bh % a.H);
-    uint16_t* dst = a.dq + (((size_t)b * a.N + n) * a.H + h) * D + c4 * 4;
+    uint16_t* dst = a.dq + b * a.dq_sb + (seq.row0 + n) * a.dq_sn + h * a.dq_sh + c4 * 4;
     uint2 w;
     w.x = pack2<BF16>(v.x * a.scale, v.y * a.scale);
     w.y = pack2<BF16>(v.z * a.scale, v.w * a.scale);
@@ -255,27 +261,50 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
 }
 
 
-// Work item (bh, key tile j); the s-th query tile it visits is tile(s). For
-// query tile i it adds into the lower sum (chain 0) when i >= j and into the
-// upper sum (chain 1) when i < j; pos(i) is its place in that chain's order
-// (0 = first, which stores instead of adding).
-// (Host-callable too, so the schedule's properties are checked on the CPU.)
+// Work items and the dQ order.
+//
+// An item is (head bh, key tile j) and runs T steps; its s-th step visits
+// query tile tile(s) = j, j+1, ..., n-1 and then (non-causal only) 0, 1, ...,
+// j-1. Items are handed out head by head, in descending j within a head.
+// Query tile i collects its dQ in two fp32 sums, each over key tiles in
+// descending j: the lower sum (chain 0) from j = i, i-1, ..., 0 and the upper
+// sum (chain 1, non-causal) from j = n-1, n-2, ..., i+1; the contributor with
+// pos(i) = 0 stores, the rest add, each after the previous one has published.
+// fa_bwd_dq adds lower + upper. The contributor a tile waits for (j + 1, same
+// head) was fetched earlier, so the earliest-fetched unfinished item never
+// waits (no deadlock), and it visited that tile one step earlier, so in
+// steady state the wait is already over. (Host-callable too, so these
+// properties are checked on the CPU.)
 struct BwdItem {
   int bh, j, T, n;
   __host__ __device__ __forceinline__ int tile(int s) const { return j + s < n ? j + s : j + s - n; }
   __host__ __device__ __forceinline__ int chain(int i) const { return i >= j ? 0 : 1; }
   __host__ __device__ __forceinline__ int pos(int i) const { return i >= j ? i - j : n - 1 - j; }
 };
-__host__ __device__ __forceinline__ BwdItem decode_item(int item, int ntiles, bool causal) {
+
+// Item number p of a launch over heads of ntiles key tiles each.
+__host__ __device__ __forceinline__ BwdItem decode_item(int p, int ntiles, bool causal) {
   BwdItem it;
-  it.bh = item / ntiles;
-  it.j = ntiles - 1 - item % ntiles;  // descending j within a head
-  it.T = causal ? ntiles - it.j : ntiles;
+  it.bh = p / ntiles;
+  it.j = ntiles - 1 - p % ntiles;  // descending j within a head
   it.n = ntiles;
+  it.T = causal ? ntiles - it.j : ntiles;
   return it;
 }
 
-template <int D, bool CAUSAL, bool BF16>
+// Item number p of this launch with its sequence's rows. A variable-length
+// sequence shorter than N has fewer key tiles (w.n); its items past them are
+// empty (T = 0) and are skipped by the producer, never handed to the roles.
+template <bool CAUSAL>
+__device__ __forceinline__ BwdItem item_of(const BwdArgs& a, int p, SeqRows* seq) {
+  BwdItem w = decode_item(p, a.ntiles, CAUSAL);
+  *seq = seq_rows(a.cu, w.bh / a.H, a.N, a.total);
+  w.n = (seq->len + 127) / 128;
+  w.T = w.j < w.n ? (CAUSAL ? w.n - w.j : w.n) : 0;
+  return w;
+}
+
+template <int D, bool CAUSAL, bool BF16, bool DROPOUT>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_dkdv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -352,12 +381,25 @@ __global__ void __launch_bounds__(512, 1)
         const int slot = n_item & 1;
         if (n_item >= 2) ok = mbar_wait(&bars->item_empty[slot], ((n_item >> 1) & 1) ^ 1, abort);
         if (!ok) break;
-        const int item = atomicAdd(a.sched, 1);
+        int item;
+        BwdItem w;
+        SeqRows seq;
+        do {  // the next item with work (empty ones exist only when variable-length)
+          item = atomicAdd(a.sched, 1);
+          if (item < total_items) w = item_of<CAUSAL>(a, item, &seq);
+        } while (item < total_items && w.T == 0);
         bars->item[slot] = item < total_items ? item : -1;
         mbar_arrive(&bars->item_full[slot]);
         if (item >= total_items) break;
-        const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
-        const int b = w.bh / a.H, h = w.bh % a.H;
+        const int b = seq.bcoord, h = w.bh % a.H;
+        const int krow = seq.row0 + w.j * 128;
+        // K_j and V_j are read from HBM once per launch; start bringing them
+        // into L2 now (the previous item still has a few steps to run), so
+        // their load below waits on L2, not on HBM.
+        for (int kb = 0; kb < D / 64; ++kb) {
+          tma_prefetch_rows(&tm_k, a.hm & kHmK, kb * 64, h, krow, b);
+          tma_prefetch_rows(&tm_v, a.hm & kHmV, kb * 64, h, krow, b);
+        }
         for (int k = 0; k < w.T && ok; ++k) {
           const int st = g % C::kStages;
           const int i = w.tile(k);
@@ -365,10 +407,10 @@ __global__ void __launch_bounds__(512, 1)
           if (!ok) break;
           mbar_arrive_expect_tx(&bars->qdo_full[st], 2 * C::kTile + 1024);
           for (int kb = 0; kb < D / 64; ++kb) {
-            tma_load_4d(&tm_q, smem + C::kQ + st * C::kTile + kb * C::kBox, &bars->qdo_full[st], kb * 64, h,
-                        i * 128, b);
-            tma_load_4d(&tm_do, smem + C::kDO + st * C::kTile + kb * C::kBox, &bars->qdo_full[st], kb * 64, h,
-                        i * 128, b);
+            tma_load_rows(&tm_q, a.hm & kHmQ, smem + C::kQ + st * C::kTile + kb * C::kBox, &bars->qdo_full[st],
+                          kb * 64, h, seq.row0 + i * 128, b);
+            tma_load_rows(&tm_do, a.hm & kHmDO, smem + C::kDO + st * C::kTile + kb * C::kBox, &bars->qdo_full[st],
+                          kb * 64, h, seq.row0 + i * 128, b);
           }
           bulk_load(smem + C::kLSE + st * 512, a.lse2 + (size_t)w.bh * a.npad + i * 128, 512, &bars->qdo_full[st]);
           bulk_load(smem + C::kDD + st * 512, a.dd + (size_t)w.bh * a.npad + i * 128, 512, &bars->qdo_full[st]);
@@ -380,8 +422,8 @@ __global__ void __launch_bounds__(512, 1)
             if (!ok) break;
             mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTile);
             for (int kb = 0; kb < D / 64; ++kb) {
-              tma_load_4d(&tm_k, smem + C::kK + kb * C::kBox, &bars->kv_full, kb * 64, h, w.j * 128, b);
-              tma_load_4d(&tm_v, smem + C::kV + kb * C::kBox, &bars->kv_full, kb * 64, h, w.j * 128, b);
+              tma_load_rows(&tm_k, a.hm & kHmK, smem + C::kK + kb * C::kBox, &bars->kv_full, kb * 64, h, krow, b);
+              tma_load_rows(&tm_v, a.hm & kHmV, smem + C::kV + kb * C::kBox, &bars->kv_full, kb * 64, h, krow, b);
             }
             ++kv_loads;
           }
@@ -425,7 +467,8 @@ __global__ void __launch_bounds__(512, 1)
         const int item = bars->item[slot];
         mbar_arrive(&bars->item_empty[slot]);
         if (item < 0) break;
-        const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
+        SeqRows seq;
+        const BwdItem w = item_of<CAUSAL>(a, item, &seq);
         ok = mbar_wait(&bars->kv_full, n_item & 1, abort) &&
              mbar_wait(&bars->qdo_full[g % C::kStages], (g / C::kStages) & 1, abort);
         if (!ok) break;
@@ -566,7 +609,8 @@ __global__ void __launch_bounds__(512, 1)
         const int item = bars->item[slot];
         mbar_arrive(&bars->item_empty[slot]);
         if (item < 0) break;
-        const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
+        SeqRows seq;
+        const BwdItem w = item_of<CAUSAL>(a, item, &seq);
         for (int k = 0; k < w.T; ++k, ++g) {
           const int i = w.tile(k);
           if (!mbar_wait(&bars->dq_added[g & 3], (g >> 2) & 1, abort)) { ok = false; break; }
@@ -601,14 +645,43 @@ __global__ void __launch_bounds__(512, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->item_empty[slot]);
       if (item < 0) break;
-      const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
+      SeqRows seq;
+      const BwdItem w = item_of<CAUSAL>(a, item, &seq);
       const int key = w.j * 128 + c;
+      // A key row past the sequence's end (the next sequence's rows when
+      // variable-length, TMA zeros otherwise) gets P = 0, so it adds nothing
+      // to dQ, and its dK, dV rows are not stored.
+      const bool key_in = key < seq.len;
       // P^T = exp2(S^T * c - LSE2) of step gs (query tile i) for this thread's
       // 64 queries, packed two per word into pk and written to TMEM over S^T
       // (columns this warpgroup has already read).
-      auto p_phase = [&](int gs, int i, uint32_t* pk) -> bool {
+      auto p_phase = [&](int gs, int i, uint32_t* pk, uint64_t& keep) -> bool {
         const int st = gs % C::kStages;
         const bool diag = CAUSAL && i == w.j;
+        if constexpr (DROPOUT) {
+          // Keep bits of this thread's key for its 64 query columns. The four
+          // lanes of a key group (keys 4g .. 4g+3) each draw one Philox call
+          // for one query of a block of four, then trade words (a 4 x 4
+          // transpose by shuffles) so that each lane holds its own key's draw
+          // for all four queries.
+          keep = 0;
+          const uint32_t grp = static_cast<uint32_t>(key) >> 2;
+          const int k4 = lane & 3;
+#pragma unroll 4
+          for (int blk = 0; blk < 16; ++blk) {
+            const uint32_t iq0 = static_cast<uint32_t>(i * 128 + wg * 64 + 4 * blk);
+            const uint4 wv = philox4x32_10(make_uint4(grp, iq0 + k4, w.bh, a.drop.offset), a.drop.seed_lo,
+                                           a.drop.seed_hi);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int idx = (k4 - q) & 3;
+              const uint32_t send = idx == 0 ? wv.x : idx == 1 ? wv.y : idx == 2 ? wv.z : wv.w;
+              const int src = (k4 + q) & 3;
+              const uint32_t got = __shfl_sync(0xffffffffu, send, (lane & ~3) | src);
+              keep |= static_cast<uint64_t>(got >= a.drop.thr ? 1u : 0u) << (4 * blk + src);
+            }
+          }
+        }
         if (!mbar_wait_warp(&bars->s_full, gs & 1, abort)) return false;
         tc_fence_after();
 #pragma unroll
@@ -623,12 +696,24 @@ __global__ void __launch_bounds__(512, 1)
             const float2 l2 = *reinterpret_cast<const float2*>(sLSE + st * 128 + qc);
             float v0 = ex2(fmaf(__uint_as_float(sv[2 * x]), cl2, -l2.x));
             float v1 = ex2(fmaf(__uint_as_float(sv[2 * x + 1]), cl2, -l2.y));
-            if (diag && key > i * 128 + qc) v0 = 0.f;
-            if (diag && key > i * 128 + qc + 1) v1 = 0.f;
+            if ((diag && key > i * 128 + qc) || !key_in) v0 = 0.f;
+            if ((diag && key > i * 128 + qc + 1) || !key_in) v1 = 0.f;
             pk[h2 * 16 + x] = pack2<BF16>(v0, v1);
           }
+          if constexpr (DROPOUT) {
+            // dV uses the dropped P (its 1 / (1 - p) is applied to dV at the
+            // end); dS below needs every P, so pk keeps them.
+            uint32_t pm[16];
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+              const int col = h2 * 32 + 2 * x;
+              pm[x] = pk[h2 * 16 + x] & (((keep >> col) & 1u ? 0x0000FFFFu : 0u) |
+                                         ((keep >> (col + 1)) & 1u ? 0xFFFF0000u : 0u));
+            }
+            tmem_st16(lane_base + C::kTS + wg * 64 + h2 * 16, pm);
+          }
         }
-        tmem_st32(lane_base + C::kTS + wg * 64, pk);
+        if constexpr (!DROPOUT) tmem_st32(lane_base + C::kTS + wg * 64, pk);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars->p_ready);
@@ -636,7 +721,7 @@ __global__ void __launch_bounds__(512, 1)
       };
       // dS^T = P^T o (dP^T - D) of step gs -> shared memory (16-bit), from the
       // same rounded P that the dV product uses.
-      auto ds_phase = [&](int gs, const uint32_t* pk) -> bool {
+      auto ds_phase = [&](int gs, const uint32_t* pk, uint64_t keep) -> bool {
         const int st = gs % C::kStages;
         if (!mbar_wait_warp(&bars->dp_full, gs & 1, abort)) return false;
         if (gs > 0 && !mbar_wait_warp(&bars->ds_free, (gs - 1) & 1, abort)) return false;
@@ -653,8 +738,15 @@ __global__ void __launch_bounds__(512, 1)
             const int qc = wg * 64 + h2 * 32 + 2 * x;
             const float2 pp = unpack2<BF16>(pk[h2 * 16 + x]);
             const float2 dd = *reinterpret_cast<const float2*>(sDD + st * 128 + qc);
-            const float d0 = pp.x * (__uint_as_float(dp[2 * x]) - dd.x);
-            const float d1 = pp.y * (__uint_as_float(dp[2 * x + 1]) - dd.y);
+            float dp0 = __uint_as_float(dp[2 * x]), dp1 = __uint_as_float(dp[2 * x + 1]);
+            if constexpr (DROPOUT) {
+              // dP = (dO V^T) o keep / (1 - p)
+              const int col = h2 * 32 + 2 * x;
+              dp0 = (keep >> col) & 1u ? dp0 * a.drop.rkeep : 0.f;
+              dp1 = (keep >> (col + 1)) & 1u ? dp1 * a.drop.rkeep : 0.f;
+            }
+            const float d0 = pp.x * (dp0 - dd.x);
+            const float d1 = pp.y * (dp1 - dd.y);
             dsk[x] = pack2<BF16>(d0, d1);
           }
           // Row c of a 128-byte-swizzled [128][64] box: 16-byte chunk x goes
@@ -676,17 +768,20 @@ __global__ void __launch_bounds__(512, 1)
       // phase earlier) and P(g+1) only waits for dV(g) and S(g+1).
       if constexpr (C::kSkew) {
         uint32_t pk_cur[32], pk_next[32];
-        if (!p_phase(g, w.tile(0), pk_cur)) { ok = false; break; }
+        uint64_t keep_cur = 0, keep_next = 0;
+        if (!p_phase(g, w.tile(0), pk_cur, keep_cur)) { ok = false; break; }
         for (int k = 0; k < w.T; ++k, ++g) {
-          if (k + 1 < w.T && !p_phase(g + 1, w.tile(k + 1), pk_next)) { ok = false; break; }
-          if (!ds_phase(g, pk_cur)) { ok = false; break; }
+          if (k + 1 < w.T && !p_phase(g + 1, w.tile(k + 1), pk_next, keep_next)) { ok = false; break; }
+          if (!ds_phase(g, pk_cur, keep_cur)) { ok = false; break; }
+          keep_cur = keep_next;
 #pragma unroll
           for (int x = 0; x < 32; ++x) pk_cur[x] = pk_next[x];
         }
       } else {
         for (int k = 0; k < w.T; ++k, ++g) {
           uint32_t pk[32];
-          if (!p_phase(g, w.tile(k), pk) || !ds_phase(g, pk)) { ok = false; break; }
+          uint64_t keep = 0;
+          if (!p_phase(g, w.tile(k), pk, keep) || !ds_phase(g, pk, keep)) { ok = false; break; }
         }
       }
       if (!ok) break;
@@ -695,9 +790,11 @@ __global__ void __launch_bounds__(512, 1)
       tc_fence_after();
       {
         const int b = w.bh / a.H, h = w.bh % a.H;
-        const bool valid = key < a.N;
-        const float mul = wg == 0 ? 1.f : a.scale;
-        uint16_t* dst = (wg == 0 ? a.dv : a.dk) + (((size_t)b * a.N + (valid ? key : 0)) * a.H + h) * D;
+        const bool valid = key_in;
+        const float mul = wg == 0 ? (DROPOUT ? a.drop.rkeep : 1.f) : a.scale;
+        const long long r = seq.row0 + (valid ? key : 0);
+        uint16_t* dst = wg == 0 ? a.dv + b * a.dv_sb + r * a.dv_sn + h * a.dv_sh
+                                : a.dk + b * a.dk_sb + r * a.dk_sn + h * a.dk_sh;
         const uint32_t src = lane_base + (wg == 0 ? C::kTdV : C::kTdK);
 #pragma unroll 1
         for (int q = 0; q < D / 32; ++q) {
@@ -712,7 +809,8 @@ __global__ void __launch_bounds__(512, 1)
           if (valid) {
             uint4* o4 = reinterpret_cast<uint4*>(dst + q * 32);
 #pragma unroll
-            for (int y = 0; y < 4; ++y) o4[y] = make_uint4(pk[4 * y], pk[4 * y + 1], pk[4 * y + 2], pk[4 * y + 3]);
+            for (int y = 0; y < 4; ++y)
+              if (q * 32 + y * 8 < a.d) o4[y] = make_uint4(pk[4 * y], pk[4 * y + 1], pk[4 * y + 2], pk[4 * y + 3]);
           }
         }
       }
@@ -737,7 +835,8 @@ __global__ void __launch_bounds__(512, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->item_empty[slot]);
       if (item < 0) break;
-      const BwdItem w = decode_item(item, a.ntiles, CAUSAL);
+      SeqRows seq;
+      const BwdItem w = item_of<CAUSAL>(a, item, &seq);
       for (int k = 0; k < w.T; ++k, ++g) {
         const int i = w.tile(k);
         // The warpgroup synchronises through two mbarriers (bounded waits, no
@@ -825,31 +924,6 @@ __global__ void __launch_bounds__(512, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-}
-
-// ------------------------------------------------------------------- launch
-
-template <int D, bool CAUSAL, bool BF16>
-cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                         const CUtensorMap& mdo, const BwdArgs& a, int num_sms, cudaStream_t s) {
-  using C = BwdCfg<D>;
-  const long long rows = (long long)a.B * a.N * a.H;
-  const int prep_blocks = (int)std::min<long long>((rows * (D / 8) + 255) / 256 + 1, 4LL * num_sms * 8);
-  fa_bwd_prep<D, BF16><<<prep_blocks, 256, 0, s>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  auto kern = fa_bwd_dkdv<D, CAUSAL, BF16>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-  if (e != cudaSuccess) return e;
-  const int items = a.B * a.H * a.ntiles;
-  const int grid = std::min(items, num_sms);
-  kern<<<grid, C::kThreads, C::kSmem, s>>>(mq, mk, mv, mdo, a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const long long dq_threads = (long long)a.B * a.H * a.npad * (D / 4);
-  const int dq_blocks = (int)std::min<long long>((dq_threads + 255) / 256, 64LL * num_sms);
-  fa_bwd_dq<D, CAUSAL, BF16><<<dq_blocks, 256, 0, s>>>(a);
-  return cudaGetLastError();
 }
 
 }  // namespace fa

@@ -207,6 +207,37 @@ __device__ __forceinline__ void tma_load_4d(const CUtensorMap* map, void* smem_d
       : "memory");
 }
 
+// Prefetch one 4-D tile into L2 (no shared-memory destination, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap* map, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+
+// A 128-row tile of a [B, N, H, d] tensor: 64 head-size columns `x`.., head h,
+// rows `row`.. of batch coordinate b. The tensor map lists its dimensions as
+// (d, H, rows, B), or as (d, rows, H, B) when the head stride exceeds the row
+// stride (head-major storage such as [B, H, N, d]); both boxes put the same
+// [128 rows][64 columns] tile into shared memory.
+__device__ __forceinline__ void tma_load_rows(const CUtensorMap* map, bool head_major, void* smem_dst,
+                                              uint64_t* bar, int x, int h, int row, int b) {
+  if (head_major)
+    tma_load_4d(map, smem_dst, bar, x, row, h, b);
+  else
+    tma_load_4d(map, smem_dst, bar, x, h, row, b);
+}
+__device__ __forceinline__ void tma_prefetch_rows(const CUtensorMap* map, bool head_major, int x, int h, int row,
+                                                  int b) {
+  if (head_major)
+    tma_prefetch_l2_4d(map, x, row, h, b);
+  else
+    tma_prefetch_l2_4d(map, x, h, row, b);
+}
+
+// Bits of FwdArgs::hm / BwdArgs::hm: which tensor maps are head-major.
+constexpr uint32_t kHmQ = 1, kHmK = 2, kHmV = 4, kHmDO = 8;
+
 // ------------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -359,6 +390,68 @@ template <int NREG, int FROM>
 __device__ __forceinline__ void reg_alloc_set() {
   if constexpr (NREG > FROM) reg_alloc_inc<NREG>();
   else if constexpr (NREG < FROM) reg_alloc_dec<NREG>();
+}
+
+// ------------------------------------------------------------ tensor layout
+
+// Rows of batch b in the caller's tensors. Fixed length (cu == nullptr): N
+// rows starting at row 0 of batch b. Variable length: cu[b] .. cu[b+1] - 1 of
+// the packed tensors (batch index 0), clamped to [0, total] and to at most N
+// rows, so a malformed offset array can shorten a sequence but never move an
+// access outside the tensors.
+struct SeqRows {
+  int row0, len, bcoord;  // first row, rows, TMA batch coordinate
+};
+__device__ __forceinline__ SeqRows seq_rows(const int* cu, int b, int N, int total) {
+  SeqRows r;
+  if (cu == nullptr) {
+    r.row0 = 0;
+    r.len = N;
+    r.bcoord = b;
+  } else {
+    int a = __ldg(cu + b), e = __ldg(cu + b + 1);
+    a = a < 0 ? 0 : (a > total ? total : a);
+    e = e < a ? a : (e > total ? total : e);
+    r.row0 = a;
+    r.len = e - a < N ? e - a : N;
+    r.bcoord = 0;
+  }
+  return r;
+}
+
+// ------------------------------------------------------------------ dropout
+
+// Philox4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel Random Numbers: As
+// Easy as 1, 2, 3", SC 2011): ten rounds of two 32x32->64-bit products with
+// the paper's multipliers, the key advanced by its Weyl constants between
+// rounds. Four 32-bit words per (counter, key).
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return c;
+}
+
+// Dropout of attention probabilities: element (query i, key j) of head
+// bh = b*H + h (b: the sequence when variable-length, i and j counted from
+// the sequence's first row) is dropped when word j % 4 of
+// philox(counter (j/4, i, bh, offset), key (seed_lo, seed_hi)) is below
+// `thr` = floor(p * 2^32). Kept values are scaled by 1 / (1 - p).
+struct Dropout {
+  uint32_t thr, seed_lo, seed_hi, offset;
+  float rkeep;  // 1 / (1 - p)
+};
+
+// Keep bits of keys 4*g .. 4*g+3 for query i (bit w = key 4g + w).
+__device__ __forceinline__ uint32_t keep4(const Dropout& dp, uint32_t g, uint32_t i, uint32_t bh) {
+  const uint4 w = philox4x32_10(make_uint4(g, i, bh, dp.offset), dp.seed_lo, dp.seed_hi);
+  return (w.x >= dp.thr ? 1u : 0u) | (w.y >= dp.thr ? 2u : 0u) | (w.z >= dp.thr ? 4u : 0u) |
+         (w.w >= dp.thr ? 8u : 0u);
 }
 
 // --------------------------------------------------------------- arithmetic

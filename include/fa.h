@@ -24,8 +24,9 @@
  *   - Layout: q, k, v, o, dout, dq, dk, dv are dense, contiguous
  *     [B, N, H, d] arrays of 16-bit floats (row stride H*d elements, head
  *     stride d). lse is a dense [B, H, N] fp32 array.
- *   - Supported: d in {64, 128}; N >= 1 of any value; B, H >= 1;
- *     B*N*H*d < 2^31. Other head sizes return FA_ERR_UNSUPPORTED.
+ *   - Supported: head size d a multiple of 8 from 8 to 128; N >= 1 of any
+ *     value; B, H >= 1; fewer than 2^31 elements per tensor. Other head
+ *     sizes return FA_ERR_UNSUPPORTED.
  *   - All pointers are DEVICE pointers on the current CUDA device, 16-byte
  *     aligned. The caller owns every buffer; the library allocates no device
  *     memory and keeps no per-call state.
@@ -33,7 +34,10 @@
  *     1/sqrt(d)).
  *   - Calls are asynchronous on `stream` and never synchronise. Arguments are
  *     checked on the host before any launch; on an error nothing is launched
- *     and no output is touched. A launch failure returns FA_ERR_CUDA.
+ *     and no output is touched. A launch whose own return code is an error
+ *     returns FA_ERR_CUDA (an error some earlier, unrelated CUDA call left
+ *     pending in the calling thread is neither reported nor cleared).
+ *     fa_last_error_detail() says which step failed and why.
  *   - Device-side waits are bounded; a wait that gives up records
  *     FA_ERR_DEVICE_TIMEOUT in a device status word that
  *     fa_check_device_status() reports.
@@ -69,6 +73,68 @@ typedef enum {
 typedef enum { FA_FP16 = 0, FA_BF16 = 1 } fa_dtype;
 
 /*
+ * Element strides of a [B, N, H, d] view of a 16-bit tensor: element
+ * (b, n, h, c) is at base[b*batch + n*row + h*head + c] (the head-size axis is
+ * contiguous). All three zero means dense [B, N, H, d]. Otherwise each must be
+ * a positive multiple of 8 elements (16 bytes) below 2^36; the batch stride
+ * may be 0 where it is never used (B = 1, or variable length). Any order of
+ * the three is accepted: e.g. a packed QKV tensor [B, N, 3, H, d] gives q, k
+ * and v the strides {N*3*H*d, 3*H*d, d} at offsets 0, H*d and 2*H*d, and
+ * PyTorch's [B, H, N, d] layout gives {H*N*d, d, N*d}.
+ */
+typedef struct {
+  long long batch, row, head;
+} fa_strides;
+
+/*
+ * One attention call's shape, options and tensor layout, for fa_fwd_ex /
+ * fa_bwd_ex. Zero-initialise it and set what is needed.
+ *   B, N, H, d       batch, sequence length, heads, head size. With
+ *                    cu_seqlens: N is the longest sequence (max_seqlen).
+ *   softmax_scale, causal, dtype   as for fa_fwd.
+ *   stride_q .. stride_dv   layout of q, k, v, o, dout, dq, dk, dv (the
+ *                    backward tensors are read only by fa_bwd_ex).
+ *   cu_seqlens       NULL: every batch entry has N rows. Otherwise a
+ *                    variable-length batch packed without padding: a device
+ *                    array of B + 1 int32 row offsets (0 = cu[0] <= cu[1] <=
+ *                    ... <= cu[B] = total), sequence b owning rows
+ *                    cu[b] .. cu[b+1]-1 of every tensor, each tensor viewed
+ *                    as [total, H, d] (batch strides unused) and lse as
+ *                    [H, total] fp32. Each sequence attends only to itself
+ *                    (causal: to its own earlier rows). The kernels clamp the
+ *                    offsets to [0, total] and lengths to N, so a malformed
+ *                    array gives wrong results, never an access outside the
+ *                    tensors.
+ *   total            rows of the packed tensors (with cu_seqlens).
+ *   dropout_p, seed, offset
+ *                    dropout on the attention probabilities (the
+ *                    dropout_p of flash_attn_func in the lab write-up §4.2
+ *                    and the README's usage line), 0 <= dropout_p < 1, 0 =
+ *                    none: O = (P o Z) V with Z = keep / (1 - dropout_p),
+ *                    the LSE that of the undropped softmax. Element (query i,
+ *                    key j) of head h of batch (or sequence) b, i and j
+ *                    counted from the sequence's first row, is dropped when
+ *                    word j mod 4 of Philox4x32-10 (Salmon et al., SC 2011)
+ *                    with counter (j / 4, i, b*H + h, offset) and key
+ *                    (seed mod 2^32, seed / 2^32) is below
+ *                    floor(dropout_p * 2^32). fa_bwd_ex regenerates the same
+ *                    mask from the same desc; nothing is stored.
+ */
+typedef struct {
+  int B, N, H, d;
+  float softmax_scale;
+  int causal;
+  fa_dtype dtype;
+  fa_strides stride_q, stride_k, stride_v, stride_o;
+  fa_strides stride_do, stride_dq, stride_dk, stride_dv;
+  const int* cu_seqlens;
+  int total;
+  float dropout_p;
+  unsigned long long seed;
+  unsigned int offset;
+} fa_desc;
+
+/*
  * Forward pass. Lab write-up §2.1 (definition), §3.1 (tiling), §3.2 (online
  * softmax with running max m and exp-sum l, rescaling of the O accumulator,
  * final O / l).
@@ -89,9 +155,28 @@ FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, fl
                  float softmax_scale, int causal, fa_dtype dtype, fa_stream_t stream);
 
 /*
+ * Forward pass on any layout fa_desc describes: strided views (e.g. the q, k
+ * and v of one packed [B, N, 3, H, d] tensor, as flash_attn_qkvpacked_func
+ * takes it in "使用FlashAttention优化PyTorch模型注意力计算", or the
+ * [B, H, N, d] layout the lab write-up §4.2 warns about), head sizes that
+ * are multiples of 8 up to 128, and variable-length batches packed without
+ * padding (the lab write-up §4.2, third pitfall: flash_attn_varlen_func).
+ * lse is dense [B, H, N] fp32, or [H, total] with cu_seqlens. Otherwise as
+ * fa_fwd.
+ */
+FA_API fa_status fa_fwd_ex(const fa_desc* desc, const void* q, const void* k, const void* v, void* o, float* lse,
+                           fa_stream_t stream);
+
+/*
  * Bytes of device workspace fa_bwd needs for this shape (0 on invalid sizes).
  * It holds D = rowsum(dO o O) [B, H, N] fp32, an fp32 dQ accumulator and the
  * per-tile ordering counters that make the dQ sum deterministic.
+ * Layout after a call (for inspection; N_pad = 128 * ceil(N / 128),
+ * up256(x) = x rounded up to a multiple of 256):
+ *   byte 0:                           LSE * log2(e), [B*H, N_pad] fp32
+ *   byte up256(4 * B*H*N_pad):        D,             [B*H, N_pad] fp32
+ *   then the dQ sums and counters (internal).
+ * Rows N .. N_pad-1 of each head hold +inf (LSE) and 0 (D).
  */
 FA_API size_t fa_bwd_workspace_size(int B, int N, int H, int d, int causal);
 
@@ -115,6 +200,20 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
                  void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int N, int H, int d,
                  float softmax_scale, int causal, fa_dtype dtype, fa_stream_t stream);
 
+/* Workspace bytes fa_bwd_ex needs for `desc` (0 if desc is invalid). */
+FA_API size_t fa_bwd_ex_workspace_size(const fa_desc* desc);
+
+/*
+ * Backward pass on any layout fa_desc describes (see fa_fwd_ex): q, k, v, o,
+ * dout, dq, dk, dv each with its own strides (dq, dk, dv may be the three
+ * slices of one packed [B, N, 3, H, d] gradient), variable-length batches,
+ * head sizes that are multiples of 8 up to 128. o and lse as fa_fwd_ex wrote
+ * them. Otherwise as fa_bwd.
+ */
+FA_API fa_status fa_bwd_ex(const fa_desc* desc, const void* q, const void* k, const void* v, const void* o,
+                           const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                           size_t workspace_bytes, fa_stream_t stream);
+
 /*
  * fa_bwd without a workspace argument, for callers that cannot allocate
  * device memory. The pages have no counterpart to this entry point.
@@ -130,8 +229,10 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
  * fa_bwd_workspace_size() exceeds that maximum returns FA_ERR_WORKSPACE and
  * launches nothing.
  *
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * Every call looks up the array's device address on the current device
+ * (cudaGetSymbolAddress; it allocates nothing, and no address is cached, so a
+ * context torn down and made again by cudaDeviceReset is handled). The first
+ * call on a device also loads this library's device code there: make that
  * first call before any stream capture. All calls on a device share the one
  * array and it keeps the last call's contents: each call re-initialises what it
  * needs (nothing has to start at zero), but calls whose work overlaps on the
@@ -143,6 +244,34 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
 FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
                                 const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int d,
                                 float softmax_scale, int causal, fa_dtype dtype, fa_stream_t stream);
+
+/*
+ * Decode step against a key/value cache (the lab write-up §6.1: inference
+ * reads a KV cache that grows one position at a time; there the work is
+ * streaming the cache, bound by memory bandwidth, not by the tensor cores).
+ *   q              in:  [B, Nq, H, d], the Nq newest positions of each
+ *                       sequence (1 <= Nq <= 8), dtype `dtype`
+ *   k_cache,
+ *   v_cache        in:  [B, Nmax, H, d]; batch b holds L_b valid rows
+ *   cache_seqlens  in:  device int32 [B], L_b (clamped to [0, Nmax]);
+ *                       rows L_b .. Nmax-1 are never read into the result
+ *                       (they may hold anything)
+ *   o              out: [B, Nq, H, d], dtype `dtype`
+ *   lse            out: [B, H, Nq] fp32
+ *   workspace      at least fa_decode_workspace_size() bytes, 16-byte
+ *                  aligned; holds each split's partial (m, l, O)
+ * Query t of batch b sits at position L_b - Nq + t; it attends keys
+ * 0 .. L_b - 1, or with causal = 1 keys 0 .. L_b - Nq + t. A row with no key
+ * to attend gets O = 0 and LSE = -inf. The cache's key axis is split across
+ * CTAs and the partial online-softmax states are merged by rescaling with
+ * the larger running max (a second launch on the same stream). All tensors
+ * dense; head size a multiple of 8 up to 128. Errors as fa_fwd; Nq > 8
+ * returns FA_ERR_UNSUPPORTED.
+ */
+FA_API size_t fa_decode_workspace_size(int B, int Nq, int H, int d, int Nmax);
+FA_API fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, const int* cache_seqlens,
+                           void* o, float* lse, void* workspace, size_t workspace_bytes, int B, int Nq, int H,
+                           int d, int Nmax, float softmax_scale, int causal, fa_dtype dtype, fa_stream_t stream);
 
 /*
  * Synchronises `stream`, then reads and clears the device status word of the
@@ -164,6 +293,25 @@ FA_API fa_status fa_check_device_status(fa_stream_t stream);
  * for other arguments, FA_ERR_CUDA if the launch fails.
  */
 FA_API fa_status fa_selftest_bounded_wait(int which, int limit_ms, fa_stream_t stream);
+
+/*
+ * Profiling hook (not part of the attention computation): after this call,
+ * every fa_bwd / fa_bwd_noalloc made from the calling host thread records
+ * `begin_event` on its stream right before the launch of its dK/dV kernel
+ * (fa_bwd_dkdv, the backward's dominant kernel) and `end_event` right after
+ * it, so cudaEventElapsedTime gives that kernel's device time. Both are
+ * cudaEvent_t handles owned by the caller; pass NULL, NULL to stop. One
+ * argument NULL and the other not returns FA_ERR_INVALID_ARG.
+ */
+FA_API fa_status fa_profile_bwd_events(void* begin_event, void* end_event);
+
+/*
+ * What the most recent call of this library from the calling host thread
+ * failed on: the step (argument check, tensor-map encoding, which launch) and,
+ * for CUDA failures, the CUDA error's name and number. Empty when that call
+ * succeeded. Thread-local storage, valid until the thread's next call.
+ */
+FA_API const char* fa_last_error_detail(void);
 
 /* Human-readable name of a status code (static storage; never NULL). */
 FA_API const char* fa_status_string(fa_status status);

@@ -60,7 +60,8 @@ def test_fwd_rejects_bad_arguments_before_launch(lib):
     assert _fwd(lib, scale=-1.0) == 1
     assert _fwd(lib, causal=2) == 1
     assert _fwd(lib, dtype=7) == 1
-    assert _fwd(lib, d=96) == 2                  # unsupported head size
+    assert _fwd(lib, d=12) == 2                  # unsupported head sizes (not a multiple of 8, > 128)
+    assert _fwd(lib, d=136) == 2
     assert _fwd(lib, d=256) == 2
     assert _fwd(lib, B=1 << 10, N=1 << 12, H=8, d=128) == 2   # >= 2^31 elements
 
@@ -68,7 +69,8 @@ def test_fwd_rejects_bad_arguments_before_launch(lib):
 def test_workspace_size(lib):
     assert fa.bwd_workspace_size(1, 1, 1, 64) > 0
     assert fa.bwd_workspace_size(0, 1, 1, 64) == 0
-    assert fa.bwd_workspace_size(1, 1, 1, 80) == 0
+    assert fa.bwd_workspace_size(1, 1, 1, 84) == 0
+    assert fa.bwd_workspace_size(1, 1, 1, 80) == fa.bwd_workspace_size(1, 1, 1, 128)
     small = fa.bwd_workspace_size(1, 128, 1, 64)
     assert fa.bwd_workspace_size(1, 256, 1, 64) > small
     assert fa.bwd_workspace_size(2, 128, 1, 64) > small
@@ -80,7 +82,7 @@ def test_bwd_rejects_bad_workspace(lib):
     need = lib.fa_bwd_workspace_size(1, 128, 1, 64, 0)
     assert lib.fa_bwd(*args, ctypes.c_void_p(0), need, 1, 128, 1, 64, 0.125, 0, 0, None) == 5
     assert lib.fa_bwd(*args, p, need - 1, 1, 128, 1, 64, 0.125, 0, 0, None) == 5
-    assert lib.fa_bwd(*args, p, need, 1, 128, 1, 48, 0.125, 0, 0, None) == 2
+    assert lib.fa_bwd(*args, p, need, 1, 128, 1, 20, 0.125, 0, 0, None) == 2
 
 
 def test_python_binding_rejects_fp32():
@@ -88,3 +90,37 @@ def test_python_binding_rejects_fp32():
     x = torch.zeros(1, 4, 1, 64)
     with pytest.raises(TypeError):
         fa.forward(x, x, x)
+
+
+def test_last_error_detail_names_the_failed_check(lib):
+    assert _fwd(lib, scale=0.0) == 1
+    assert "softmax_scale" in fa.last_error_detail()
+    assert _fwd(lib, d=100) == 2
+    assert "head_dim" in fa.last_error_detail()
+    assert _fwd(lib, ptr=8) == 1
+    assert "aligned" in fa.last_error_detail()
+
+
+def test_profile_hook_needs_both_events_or_neither(lib):
+    assert lib.fa_profile_bwd_events(ctypes.c_void_p(16), None) == 1
+    assert lib.fa_profile_bwd_events(None, ctypes.c_void_p(16)) == 1
+    assert lib.fa_profile_bwd_events(None, None) == 0
+
+
+class _OnDevice:
+    def __init__(self, device):
+        self.device = device
+
+
+def test_binding_rejects_tensors_and_streams_on_another_device():
+    # forward/backward run on q's device; anything else the call would touch
+    # (lse, outputs, workspace, stream) must be on that device too.
+    import torch
+    d0, d1 = torch.device("cuda", 0), torch.device("cuda", 1)
+    fa.check_same_device(d0, lse=_OnDevice(d0), stream=_OnDevice(d0), workspace=None)
+    with pytest.raises(ValueError, match="lse"):
+        fa.check_same_device(d0, lse=_OnDevice(d1))
+    with pytest.raises(ValueError, match="stream"):
+        fa.check_same_device(d0, lse=_OnDevice(d0), stream=_OnDevice(d1))
+    with pytest.raises(ValueError, match="workspace"):
+        fa.check_same_device(d1, workspace=_OnDevice(d0))

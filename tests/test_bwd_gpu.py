@@ -139,7 +139,7 @@ def test_autograd_wrapper_matches_direct_calls(causal):
     case = Case(1, 300, 2, 64, "fp16", causal, seed=3)
     q, k, v, do = (case.torch(n) for n in ("q", "k", "v", "do"))
     qr, kr, vr = (t.clone().requires_grad_(True) for t in (q, k, v))
-    y = fa.flash_attn_func(qr, kr, vr, case.scale, causal)
+    y = fa.flash_attn_func(qr, kr, vr, 0.0, case.scale, causal)
     y.backward(do)
     o, lse = fa.forward(q, k, v, case.scale, causal)
     dq, dk, dv = fa.backward(q, k, v, o, do, lse, case.scale, causal)
@@ -147,3 +147,51 @@ def test_autograd_wrapper_matches_direct_calls(causal):
     assert torch.equal(y.detach(), o)
     for got, want in ((qr.grad, dq), (kr.grad, dk), (vr.grad, dv)):
         assert torch.equal(got, want)
+
+
+def _workspace_d(ws, B, N, H):
+    """D = rowsum(dO o O) as fa_bwd left it in the workspace: [B*H, N_pad]
+    fp32 at byte offset up256(4 * B*H*N_pad) (the layout include/fa.h states)."""
+    npad = 128 * ((N + 127) // 128)
+    off = (4 * B * H * npad + 255) // 256 * 256
+    raw = ws[off:off + 4 * B * H * npad].view(torch.float32).view(B * H, npad)
+    return raw.double().cpu().numpy(), npad
+
+
+@pytest.mark.parametrize("B,N,H,d,dtype,causal", [
+    (1, 300, 2, 64, "fp16", False),
+    (2, 1000, 3, 128, "bf16", True),
+    (4, 4096, 8, 128, "bf16", True),
+])
+def test_preprocess_d_matches_its_definition_and_the_oracle(B, N, H, d, dtype, causal):
+    # D is computed by the preprocessing kernel from the forward's (rounded)
+    # O and dO. Against rowsum(dO o O) of the same O in fp64, only fp32
+    # accumulation error remains (a few ulps of sum |dO o O|). Against the
+    # oracle's D (exact O), the gap is bounded by sum_k |dO_ik| * max|O_gpu -
+    # O_exact|, which the forward's own O error gives.
+    import exact_attention_119_b200 as fa
+    from oracle import attention_forward
+    case = Case(B, N, H, d, dtype, causal, seed=31)
+    q, k, v, do = (case.torch(n) for n in ("q", "k", "v", "do"))
+    o, lse = fa.forward(q, k, v, case.scale, causal)
+    ws = torch.zeros(fa.bwd_workspace_size(B, N, H, d, causal), dtype=torch.uint8, device="cuda")
+    fa.backward(q, k, v, o, do, lse, case.scale, causal, workspace=ws)
+    assert fa.check_device_status() == 0
+    dd, npad = _workspace_d(ws, B, N, H)
+    og = o.double().cpu().numpy()
+    dof = case.f64["do"]
+    prod = dof * og                                        # [B, N, H, d]
+    want = prod.sum(axis=3).transpose(0, 2, 1).reshape(B * H, N)
+    mag = np.abs(prod).sum(axis=3).transpose(0, 2, 1).reshape(B * H, N)
+    got = dd[:, :N]
+    assert np.all(np.abs(got - want) <= 1e-5 * mag + 1e-6)
+    assert np.all(dd[:, N:] == 0.0)                        # pad rows
+    # against the oracle (heads sampled at the large size)
+    heads = [(0, 0), (B - 1, H - 1)] if N >= 4096 else None
+    ro, _ = attention_forward(case.f64["q"], case.f64["k"], case.f64["v"], case.scale, causal)
+    _, _, _, rd = attention_backward(case.f64["q"], case.f64["k"], case.f64["v"], dof, case.scale, causal,
+                                     heads=heads)
+    for b, h in heads or [(b, h) for b in range(B) for h in range(H)]:
+        o_err = np.abs(og[b, :, h] - ro[b, :, h]).max()
+        bound = np.abs(dof[b, :, h]).sum(axis=1) * o_err + 1e-5 * mag[b * H + h] + 1e-6
+        assert np.all(np.abs(got[b * H + h] - rd[b, h]) <= bound), (b, h)

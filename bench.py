@@ -3,12 +3,15 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 One step = one fa_fwd + one fa_bwd over one batch of the workload (the whole
-hot path). Timing: CUDA events on the launching stream around each step, L2
-flushed (256 MiB write) before every step and the flush excluded; the K timed
-steps are bracketed by a barrier and a device synchronize on both sides and
-the time is the max over ranks. Multi-GPU (torchrun): every rank runs its own
-independent batch (attention heads share nothing), no collective on the data
-path, weak scaling.
+hot path). The default workload is the 12-layer decoder's attention: B=4,
+N=4096, H=8, d=128, bf16, causal. Timing: CUDA events on the launching stream
+around each call, and around the backward's dK/dV kernel itself (the
+library's profiling hook); L2 flushed (256 MiB write) before every step, the
+flush not timed; the K timed steps are bracketed by a barrier and a device
+synchronize on both sides and the time is the max over ranks. SM clocks and
+throttle reasons are polled through NVML every 2 ms while the timed steps run.
+Multi-GPU (torchrun): every rank runs its own independent batch (attention
+heads share nothing), no collective on the data path, weak scaling.
 
 Metric: fwd+bwd TFLOPS with counted FLOPs 4*B*H*N^2*d (fwd) + 10*B*H*N^2*d
 (bwd), halved when causal; fwd-only TFLOPS is reported beside it.
@@ -25,7 +28,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -45,14 +47,46 @@ WORKLOADS = {
 for _n in (512, 1024, 2048, 4096, 8192, 16384, 32768):
     for _c in (False, True):
         WORKLOADS[f"sweep_N{_n}_H16_d128_bf16{'_causal' if _c else ''}"] = (max(1, 16384 // _n), _n, 16, 128, "bf16", _c)
-DEFAULT_WORKLOAD = "p4_B2_N2048_H12_d64_fp16"
+DEFAULT_WORKLOAD = "decoder_B4_N4096_H8_d128_bf16_causal"
 
-# ncu DRAM bytes per launch of the dominant kernel, from the capture summarised
-# in profiles/ for the default workload; None when the kernel has changed since.
-NCU_TRAFFIC_BYTES = {
-    # fa_bwd_dkdv<64,0,0>: dram__bytes_read.sum 25,630,976 + dram__bytes_write.sum 304,384
-    ("p4_B2_N2048_H12_d64_fp16", "fa_bwd_dkdv"): 25_935_360,
+# Kernel sources whose hash keys a committed ncu traffic figure: a figure
+# taken from an older version of the kernel is not reported.
+KERNEL_SOURCES = {
+    "fa_bwd_dkdv": ["sm100.cuh", "bwd_kernels.cuh"],
+    "fa_fwd_kernel": ["sm100.cuh", "fwd_kernel.cuh"],
 }
+
+
+def sources_sha256(kernel):
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "exact_attention_119_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload, kernel):
+    """DRAM bytes per launch of `kernel` on `workload` from the ncu summaries
+    under profiles/ (a line 'bench-key: workload=W kernel=K traffic_bytes=T
+    sources_sha256=S'); (bytes, note). Null when no summary matches or the
+    kernel source has changed since the capture."""
+    import glob
+    import re
+    want = sources_sha256(kernel)
+    stale = None
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        with open(path) as f:
+            for line in f:
+                m = re.search(r"bench-key: workload=(\S+) kernel=(\S+) traffic_bytes=(\d+) sources_sha256=(\w+)", line)
+                if m and m.group(1) == workload and m.group(2) == kernel:
+                    if m.group(4) == want:
+                        return int(m.group(3)), f"ncu capture in profiles/{os.path.basename(path)}"
+                    stale = os.path.basename(path)
+    if stale:
+        return None, f"profiles/{stale} was captured from an older kernel source (stale)"
+    return None, "no ncu capture of this kernel and workload under profiles/"
+
 
 SPEC_TFLOPS = 2250.0  # nominal dense fp16/bf16 tensor rate of one B200
 
@@ -85,70 +119,65 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+    """SM clock, power and throttle reasons polled through NVML every 2 ms on
+    a host thread while the timed steps run (nvidia-smi -lms 50 is the
+    fallback); only samples inside the marked window count."""
 
-    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
     def __init__(self, index):
         self.index = index
-        self.proc = None
-        self.path = None
+        self.samples = []
         self.window = None
+        self._stop = None
+        self._thread = None
+        self._nvml = None
 
     def start(self):
-        """Start sampling every 50 ms; give nvidia-smi a head start."""
+        import threading
         try:
-            import tempfile
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-            time.sleep(0.5)
-        except OSError:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            handle = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self._nvml = pynvml
+        except Exception:  # no NVML: no samples, the line says so
+            return
+        self._stop = threading.Event()
+
+        def poll():
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            while not self._stop.is_set():
+                try:
+                    sm = pynvml.nvmlDeviceGetClockInfo(handle, pynvml.NVML_CLOCK_SM)
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                    pw = pynvml.nvmlDeviceGetPowerUsage(handle) / 1000.0
+                    self.samples.append((time.time(), sm, mx, rs, pw))
+                except Exception:
+                    pass
+                time.sleep(0.002)
+
+        self._thread = threading.Thread(target=poll, daemon=True)
+        self._thread.start()
+        time.sleep(0.05)
 
     def mark(self, t0, t1):
         """Host wall-clock bounds of the timed region."""
         self.window = (t0, t1)
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        import datetime
-        sms, maxes, reasons, total = [], [], set(), 0
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                cols = [c.strip() for c in line.split(",")]
-                if len(cols) < 10:
-                    continue
-                try:
-                    ts = datetime.datetime.strptime(cols[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
-                    sm, mx = float(cols[2]), float(cols[3])
-                except ValueError:
-                    continue
-                total += 1
-                if self.window and not (self.window[0] <= ts <= self.window[1]):
-                    continue
-                sms.append(sm)
-                maxes.append(mx)
-                for name, val in zip(names, cols[6:10]):
-                    if val.lower() == "active":
-                        reasons.add(name)
-        os.unlink(self.path)
-        if not sms:
+        if self._thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "note": "NVML unavailable"}
+        self._stop.set()
+        self._thread.join(timeout=5)
+        inside = [x for x in self.samples if self.window and self.window[0] <= x[0] <= self.window[1]]
+        if not inside:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
-                    "note": f"no sample inside the timed window ({total} outside)"}
-        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes), "reasons": sorted(reasons),
-                "samples": len(sms)}
+                    "note": f"no sample inside the timed window ({len(self.samples)} outside)"}
+        reasons = sorted({name for x in inside for name, bit in self.REASONS.items() if x[3] & bit})
+        return {"sm_mhz": statistics.median(x[1] for x in inside), "sm_max_mhz": max(x[2] for x in inside),
+                "sm_min_mhz": min(x[1] for x in inside), "power_w_median": statistics.median(x[4] for x in inside),
+                "reasons": reasons, "samples": len(inside), "source": "NVML, 2 ms polling"}
 
 
 def dist_env():
@@ -228,49 +257,160 @@ def run_reference(args, workload):
     return 0
 
 
-EXTRA_WORKLOADS = ["decoder_B4_N4096_H8_d128_bf16_causal", "llama7b_B1_N4096_H32_d128_bf16_causal",
-                   "sweep_N4096_H16_d128_bf16", "sweep_N16384_H16_d128_bf16"]
+# Reported beside the headline, same protocol, fewer steps: the other
+# workloads the stated targets are quoted on (N >= 4096, d = 128) and the
+# pages' d = 64 comparison shape.
+EXTRA_WORKLOADS = ["llama7b_B1_N4096_H32_d128_bf16_causal", "sweep_N4096_H16_d128_bf16",
+                   "sweep_N16384_H16_d128_bf16", "sweep_N16384_H16_d128_bf16_causal", "p4_B2_N2048_H12_d64_fp16"]
+
+
+class Buffers:
+    """Device inputs and outputs of one workload (inputs seeded on the host)."""
+
+    def __init__(self, workload, dev, rank, pinned=False):
+        import torch
+        import exact_attention_119_b200 as fa
+        from exact_attention_119_b200 import inputs
+        B, N, H, d, dtype, causal = workload
+        self.workload = workload
+        self.scale = 1.0 / math.sqrt(d)
+        bits = inputs.attention_inputs(B, N, H, d, dtype, seed=rank)
+        self.host = {k: inputs.bits_to_torch(v, dtype) for k, v in bits.items()}
+        if pinned:
+            self.host = {k: v.pin_memory() for k, v in self.host.items()}
+        self.q, self.k, self.v, self.do = (self.host[n].to(dev) for n in ("q", "k", "v", "do"))
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        self.dq, self.dk, self.dv = (torch.empty_like(self.q) for _ in range(3))
+        self.ws = torch.empty(max(16, fa.bwd_workspace_size(B, N, H, d, causal)), dtype=torch.uint8, device=dev)
+
+    def fwd(self):
+        import exact_attention_119_b200 as fa
+        fa.forward(self.q, self.k, self.v, self.scale, self.workload[5], out=self.o, lse=self.lse)
+
+    def bwd(self):
+        import exact_attention_119_b200 as fa
+        fa.backward(self.q, self.k, self.v, self.o, self.do, self.lse, self.scale, self.workload[5],
+                    self.dq, self.dk, self.dv, workspace=self.ws)
+
+
+def timed_steps(buf, steps, stream, flush):
+    """Run `steps` steps with events around fa_fwd, fa_bwd and the backward's
+    dK/dV kernel; returns per-step (fwd, bwd, dkdv) milliseconds. The L2 is
+    flushed before each step unless flush is None."""
+    import torch
+    import exact_attention_119_b200 as fa
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    for i in range(steps):
+        if flush is not None:
+            flush.fill_(i & 0xFF)
+        fa.profile_bwd_events(ev[i][3], ev[i][4])
+        ev[i][0].record(stream)
+        buf.fwd()
+        ev[i][1].record(stream)
+        buf.bwd()
+        ev[i][2].record(stream)
+    fa.profile_bwd_events(None, None)
+    return ev
+
+
+def elapsed(ev):
+    return ([e[0].elapsed_time(e[1]) for e in ev], [e[1].elapsed_time(e[2]) for e in ev],
+            [e[3].elapsed_time(e[4]) for e in ev])
 
 
 def time_workload(workload, steps, warmup, dev, stream, flush, world, rank):
-    """fwd, bwd and fwd+bwd TFLOPS of one workload (events per call, L2 flushed)."""
+    """fwd, bwd, fwd+bwd and dK/dV-kernel TFLOPS of one workload (events per
+    call, L2 flushed)."""
     import torch
     import exact_attention_119_b200 as fa
-    from exact_attention_119_b200 import inputs
-    B, N, H, d, dtype, causal = workload
-    scale = 1.0 / math.sqrt(d)
-    bits = inputs.attention_inputs(B, N, H, d, dtype, seed=rank)
-    q, k, v, do = (inputs.bits_to_torch(bits[n], dtype).to(dev) for n in ("q", "k", "v", "do"))
-    o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
-    ws = torch.empty(max(16, fa.bwd_workspace_size(B, N, H, d, causal)), dtype=torch.uint8, device=dev)
+    buf = Buffers(workload, dev, rank)
     for _ in range(warmup):
-        fa.forward(q, k, v, scale, causal, out=o, lse=lse)
-        fa.backward(q, k, v, o, do, lse, scale, causal, dq, dk, dv, workspace=ws)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        buf.fwd()
+        buf.bwd()
     torch.cuda.synchronize(dev)
-    for i in range(steps):
-        flush.fill_(i & 0xFF)
-        ev[i][0].record(stream)
-        fa.forward(q, k, v, scale, causal, out=o, lse=lse)
-        ev[i][1].record(stream)
-        fa.backward(q, k, v, o, do, lse, scale, causal, dq, dk, dv, workspace=ws)
-        ev[i][2].record(stream)
+    ev = timed_steps(buf, steps, stream, flush)
     torch.cuda.synchronize(dev)
     if fa.check_device_status() != 0:
         raise RuntimeError("device status not OK")
-    f_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
-    b_ms = sum(e[1].elapsed_time(e[2]) for e in ev)
-    f_ms, b_ms = reduce_max([f_ms, b_ms], world, dev)
+    f, b, k = (sum(x) for x in elapsed(ev))
+    f_ms, b_ms, k_ms = reduce_max([f, b, k], world, dev)
+    B, N, H, d, dtype, causal = workload
     f_fwd, f_bwd = flops(B, N, H, d, causal)
     out = {"fwd_tflops": whole_job_tflops(world, steps, f_fwd, f_ms),
            "bwd_tflops": whole_job_tflops(world, steps, f_bwd, b_ms),
            "fwd_bwd_tflops": whole_job_tflops(world, steps, f_fwd + f_bwd, f_ms + b_ms),
+           "dkdv_kernel_tflops": whole_job_tflops(world, steps, f_bwd, k_ms),
            "steps": steps}
-    del q, k, v, do, o, lse, dq, dk, dv, ws
+    del buf
     torch.cuda.empty_cache()
     return out
+
+
+# KV-cache decode (one new position per sequence against a long cache): an
+# HBM-bound workload, reported as GB/s of cache read against the HBM peak.
+DECODE_WORKLOADS = {
+    "decode_B8_H32_L8192_d128_bf16": (8, 1, 32, 128, 8192, "bf16"),
+    "decode_B1_H32_L32768_d128_bf16": (1, 1, 32, 128, 32768, "bf16"),
+}
+
+
+def time_decode(workload, steps, dev, stream, flush, world, rank):
+    """fa_decode over a full cache: device time per call (events, L2 flushed
+    before each call), and the cache bytes it must read per call."""
+    import torch
+    import exact_attention_119_b200 as fa
+    from exact_attention_119_b200 import inputs
+    B, Nq, H, d, L, dtype = workload
+    q = inputs.bits_to_torch(inputs.make_tensor_bits((B, Nq, H, d), dtype, rank, 0), dtype).to(dev)
+    kc = inputs.bits_to_torch(inputs.make_tensor_bits((B, L, H, d), dtype, rank, 1), dtype).to(dev)
+    vc = inputs.bits_to_torch(inputs.make_tensor_bits((B, L, H, d), dtype, rank, 2), dtype).to(dev)
+    lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(16, fa.decode_workspace_size(B, Nq, H, d, L)), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        fa.decode(q, kc, vc, lens, None, False, out=o, lse=lse, workspace=ws)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        fa.decode(q, kc, vc, lens, None, False, out=o, lse=lse, workspace=ws)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    if fa.check_device_status() != 0:
+        raise RuntimeError("device status not OK")
+    (ms,) = reduce_max([sum(a.elapsed_time(b) for a, b in ev)], world, dev)
+    nbytes = 2 * B * L * H * d * 2 + 2 * B * Nq * H * d * 2 + B * H * Nq * 4
+    out = {"us_per_call": 1e3 * ms / steps, "gbs": world * steps * nbytes / (ms * 1e-3) / 1e9,
+           "bytes_per_call": nbytes, "steps": steps,
+           "note": "K and V cache read once, q read, O and LSE written (the partial states stay in L2)"}
+    del q, kc, vc, o, lse, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_decode_only(args):
+    """--workload decode_*: only the KV-cache decode, as GB/s of cache read
+    (a side measurement; the headline is the attention fwd+bwd step)."""
+    import torch
+    world, rank, local = dist_env()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    if args.impl == "reference":
+        print(json.dumps({"impl": "reference", "unavailable": "the decode side measurement has no reference arm"}))
+        return 0
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    r = time_decode(DECODE_WORKLOADS[args.workload], args.steps, dev, torch.cuda.current_stream(dev), flush, 1, 0)
+    peaks, kind = load_peaks()
+    B, Nq, H, d, L, dtype = DECODE_WORKLOADS[args.workload]
+    print(json.dumps({"metric": "KV-cache decode GB/s", "value": r["gbs"], "unit": "GB/s", "n_gpus": 1,
+                      "steps": args.steps, "higher_is_better": True, "dtype": dtype,
+                      "config": {"workload": args.workload, "batch": B, "new_rows": Nq, "heads": H, "head_dim": d,
+                                 "cache_len": L},
+                      "frac_of_hbm_peak": r["gbs"] / float(peaks["hbm_gbs"]), "peak_kind": kind, **r}))
+    return 0
 
 
 def config_dict(name, workload):
@@ -283,17 +423,19 @@ def config_dict(name, workload):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
-                    help="skip the N>=4096, d=128 workloads reported beside the default one")
+                    help="skip the other workloads reported beside the headline")
     ap.add_argument("--extra-steps", type=int, default=30)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload in DECODE_WORKLOADS:
+        return run_decode_only(args)
     workload = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, workload)
@@ -302,7 +444,6 @@ def main():
     import torch.distributed as dist
 
     import exact_attention_119_b200 as fa
-    from exact_attention_119_b200 import inputs
 
     world, rank, local = dist_env()
     if world > 1:
@@ -313,41 +454,25 @@ def main():
     torch.cuda.set_device(dev)
 
     B, N, H, d, dtype, causal = workload
-    scale = 1.0 / math.sqrt(d)
-    bits = inputs.attention_inputs(B, N, H, d, dtype, seed=rank)
-    host = {k: inputs.bits_to_torch(v, dtype).pin_memory() for k, v in bits.items()}
-    q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "do"))
-    o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
-    ws = torch.empty(max(16, fa.bwd_workspace_size(B, N, H, d, causal)), dtype=torch.uint8, device=dev)
+    buf = Buffers(workload, dev, rank, pinned=True)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        fa.forward(q, k, v, scale, causal, out=o, lse=lse)
-        fa.backward(q, k, v, o, do, lse, scale, causal, dq, dk, dv, workspace=ws)
-
     for _ in range(args.warmup):
         flush.fill_(1)
-        step()
+        buf.fwd()
+        buf.bwd()
     torch.cuda.synchronize(dev)
     assert fa.check_device_status() == 0
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    # ---- the timed steps (device-resident inputs)
     sampler = ClockSampler(dev.index)
     sampler.start()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        ev[i][0].record(stream)
-        fa.forward(q, k, v, scale, causal, out=o, lse=lse)
-        ev[i][1].record(stream)
-        fa.backward(q, k, v, o, do, lse, scale, causal, dq, dk, dv, workspace=ws)
-        ev[i][2].record(stream)
+    ev = timed_steps(buf, args.steps, stream, flush)
     torch.cuda.synchronize(dev)
     sampler.mark(t_wall0, time.time())
     if world > 1:
@@ -356,18 +481,19 @@ def main():
     status = fa.check_device_status()
     if status != 0:
         raise RuntimeError(f"device status {fa.status_string(status)} after the timed steps")
-    fwd_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    bwd_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    tot_ms = sum(fwd_ms) + sum(bwd_ms)
-    tot_ms, fwd_sum, bwd_sum = reduce_max([tot_ms, sum(fwd_ms), sum(bwd_ms)], world, dev)
+    fwd_ms, bwd_ms, dkdv_ms = elapsed(ev)
+    tot_ms, fwd_sum, bwd_sum, dkdv_sum = reduce_max(
+        [sum(fwd_ms) + sum(bwd_ms), sum(fwd_ms), sum(bwd_ms), sum(dkdv_ms)], world, dev)
 
     f_fwd, f_bwd = flops(B, N, H, d, causal)
     value = whole_job_tflops(world, args.steps, f_fwd + f_bwd, tot_ms)
     fwd_tflops = whole_job_tflops(world, args.steps, f_fwd, fwd_sum)
     bwd_tflops = whole_job_tflops(world, args.steps, f_bwd, bwd_sum)
+    dkdv_tflops = whole_job_tflops(world, args.steps, f_bwd, dkdv_sum)
 
     # ---- end to end through the public API: pinned host in, results back out
-    out_host = {n: torch.empty_like(host["q"]).pin_memory() for n in ("o", "dq", "dk", "dv")}
+    q, k, v, do = buf.q, buf.k, buf.v, buf.do
+    out_host = {n: torch.empty_like(buf.host["q"]).pin_memory() for n in ("o", "dq", "dk", "dv")}
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
@@ -375,15 +501,16 @@ def main():
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
         e2e_ev[i][0].record(stream)
-        q.copy_(host["q"], non_blocking=True)
-        k.copy_(host["k"], non_blocking=True)
-        v.copy_(host["v"], non_blocking=True)
-        do.copy_(host["do"], non_blocking=True)
-        step()
-        out_host["o"].copy_(o, non_blocking=True)
-        out_host["dq"].copy_(dq, non_blocking=True)
-        out_host["dk"].copy_(dk, non_blocking=True)
-        out_host["dv"].copy_(dv, non_blocking=True)
+        q.copy_(buf.host["q"], non_blocking=True)
+        k.copy_(buf.host["k"], non_blocking=True)
+        v.copy_(buf.host["v"], non_blocking=True)
+        do.copy_(buf.host["do"], non_blocking=True)
+        buf.fwd()
+        buf.bwd()
+        out_host["o"].copy_(buf.o, non_blocking=True)
+        out_host["dq"].copy_(buf.dq, non_blocking=True)
+        out_host["dk"].copy_(buf.dk, non_blocking=True)
+        out_host["dv"].copy_(buf.dv, non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     (e2e_ms,) = reduce_max([sum(a.elapsed_time(b) for a, b in e2e_ev)], world, dev)
@@ -393,19 +520,13 @@ def main():
     tensor_bytes = B * N * H * d * 2
 
     # ---- the same steps back to back without the L2 flush, reported beside the headline
-    nf_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    for i in range(args.steps):
-        nf_ev[i][0].record(stream)
-        fa.forward(q, k, v, scale, causal, out=o, lse=lse)
-        nf_ev[i][1].record(stream)
-        fa.backward(q, k, v, o, do, lse, scale, causal, dq, dk, dv, workspace=ws)
-        nf_ev[i][2].record(stream)
+    nf = timed_steps(buf, args.steps, stream, None)
     torch.cuda.synchronize(dev)
-    nf_f, nf_b = reduce_max([sum(e[0].elapsed_time(e[1]) for e in nf_ev), sum(e[1].elapsed_time(e[2]) for e in nf_ev)],
-                            world, dev)
+    nf_f, nf_b, _ = (sum(x) for x in elapsed(nf))
+    nf_f, nf_b = reduce_max([nf_f, nf_b], world, dev)
     if world > 1:
         dist.barrier()
     no_flush = {"value": whole_job_tflops(world, args.steps, f_fwd + f_bwd, nf_f + nf_b),
@@ -414,17 +535,17 @@ def main():
                 "note": "the same steps back to back, L2 not flushed between them"}
 
     peaks, peak_kind = load_peaks()
-    peak = float(peaks["bf16_tflops"])  # fp16 and bf16 run at the same dense tensor rate
-    dominant = "fa_bwd_dkdv" if bwd_sum >= fwd_sum else "fa_fwd"
-    achieved = bwd_tflops if dominant == "fa_bwd_dkdv" else fwd_tflops
-    traffic = NCU_TRAFFIC_BYTES.get((args.workload, dominant))
+    # fp16 and bf16 run at the same dense tensor rate. A kernel timed inside a
+    # step of a few hundred microseconds is a burst, not a seconds-long loop.
+    peak = float(peaks["bf16_tflops"])
+    traffic, traffic_note = committed_traffic(args.workload, "fa_bwd_dkdv")
 
-    # ---- the workloads the stated targets are quoted on (N >= 4096, d = 128):
-    # same timing protocol, fewer steps, reported beside the headline.
-    extra = {}
+    extra, decode = {}, {}
     if not args.no_extra and args.workload == DEFAULT_WORKLOAD:
         for name in EXTRA_WORKLOADS:
             extra[name] = time_workload(WORKLOADS[name], args.extra_steps, 3, dev, stream, flush, world, rank)
+        for name, wl in DECODE_WORKLOADS.items():
+            decode[name] = time_decode(wl, 50, dev, stream, flush, world, rank)
 
     if rank == 0:
         line = {
@@ -433,16 +554,23 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "f16" if dtype == "fp16" else "bf16",
             "data": "synthetic", "config": config_dict(args.workload, workload),
             "fwd_tflops": fwd_tflops, "bwd_tflops": bwd_tflops,
-            "fwd_ms": fwd_sum / args.steps, "bwd_ms": bwd_sum / args.steps,
+            "fwd_ms": fwd_sum / args.steps, "bwd_ms": bwd_sum / args.steps, "dkdv_kernel_ms": dkdv_sum / args.steps,
             "frac_of_peak": {"fwd": fwd_tflops / world / peak, "fwd_bwd": value / world / peak,
                              "peak_tflops": peak, "peak_kind": peak_kind + " bf16 dense (cuBLAS burst)",
                              "fwd_spec": fwd_tflops / world / SPEC_TFLOPS, "fwd_bwd_spec": value / world / SPEC_TFLOPS,
                              "spec_tflops": SPEC_TFLOPS},
             "no_l2_flush": no_flush,
-            "roofline": {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                         "note": ("fa_bwd timed as one call: prep + dkdv + dq launches" if dominant == "fa_bwd_dkdv"
-                                  else "one launch per call") + f"; peak {peak_kind}"},
+            "roofline": {"bound": "tensor", "kernel": "fa_bwd_dkdv", "achieved": dkdv_tflops / world, "peak": peak,
+                         "unit": "TFLOP/s", "frac": dkdv_tflops / world / peak, "traffic": traffic,
+                         "note": ("the backward's dK/dV kernel, which runs all five backward contractions "
+                                  "(10*B*H*N^2*d, halved when causal), timed by events on its own launch; "
+                                  f"peak {peak_kind}; traffic: {traffic_note}")},
+            "kernels": {
+                "fa_fwd_kernel": {"tflops": fwd_tflops / world, "frac": fwd_tflops / world / peak,
+                                  "ms": fwd_sum / args.steps},
+                "fa_bwd_dkdv": {"tflops": dkdv_tflops / world, "frac": dkdv_tflops / world / peak,
+                                "ms": dkdv_sum / args.steps},
+                "fa_bwd_prep+fa_bwd_dq": {"ms": (bwd_sum - dkdv_sum) / args.steps}},
             "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": 4 * tensor_bytes,
                     "d2h_bytes_per_step": 4 * tensor_bytes},
             "gpu_launches": 4 * args.steps,
@@ -464,7 +592,14 @@ def main():
             for v in extra.values():
                 v["fwd_frac_of_peak"] = v["fwd_tflops"] / peak
                 v["fwd_bwd_frac_of_peak"] = v["fwd_bwd_tflops"] / peak
-            line["target_workloads"] = extra
+                v["dkdv_frac_of_peak"] = v["dkdv_kernel_tflops"] / peak
+            line["other_workloads"] = extra
+        if decode:
+            hbm = float(peaks["hbm_gbs"])
+            for v in decode.values():
+                v["frac_of_hbm_peak"] = v["gbs"] / world / hbm
+                v["hbm_peak_gbs"] = hbm
+            line["decode_workloads"] = decode
         if world == 1 and not args.no_cpu_baseline:
             smp = oracle_sample(workload, budget_s=15.0)
             line["cpu_baseline"] = {

@@ -93,85 +93,104 @@ struct BwdArgs {
 
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256) fa_bwd_prep(const BwdArgs a) {
-  // A group of G = D/8 lanes per (b, h, n) row, 8 elements per lane, over
-  // n < npad of every head: rows of the sequence get D = rowsum(dO o O) and
-  // LSE*log2(e); rows past its end get 0 and +inf (no query: P = 0).
+  // Block (x, bh): rows n = x * kRows + group of head bh, a group of G = D/8
+  // lanes per row, 8 elements per lane. Rows of the sequence get
+  // D = rowsum(dO o O) and LSE*log2(e); rows past its end (up to npad) get 0
+  // and +inf (no query: P = 0).
   constexpr int G = D / 8;
-  const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-  const long long nthreads = (long long)gridDim.x * blockDim.x;
-  const long long rows = (long long)a.B * a.H * a.npad;
-  const int lane = threadIdx.x & 31;
-  const int sub = lane % G;
-  const long long ngroups = nthreads / G;
-  for (long long row0 = (tid / 32) * (32 / G); row0 < rows; row0 += ngroups) {
-    const long long row = row0 + lane / G;  // bh * npad + n
-    const bool in = row < rows;
-    const int bh = in ? (int)(row / a.npad) : 0;
-    const int n = in ? (int)(row % a.npad) : 0;
-    const int b = bh / a.H, h = bh % a.H;
-    const SeqRows seq = seq_rows(a.cu, b, a.N, a.total);
-    const bool valid = in && n < seq.len;
-    float acc = 0.f;
-    if (valid && sub * 8 < a.d) {
-      const long long r = seq.row0 + n;
-      const uint4 ov = *reinterpret_cast<const uint4*>(a.o + b * a.o_sb + r * a.o_sn + h * a.o_sh + sub * 8);
-      const uint4 dv = *reinterpret_cast<const uint4*>(a.dout + b * a.do_sb + r * a.do_sn + h * a.do_sh + sub * 8);
-      const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
-      const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
+  constexpr int kRows = 256 / G;
+  const int bh = blockIdx.y;
+  const int b = bh / a.H, h = bh % a.H;
+  const int sub = threadIdx.x % G;
+  const int n = blockIdx.x * kRows + threadIdx.x / G;
+  const SeqRows seq = seq_rows(a.cu, b, a.N, a.total);
+  const bool valid = n < seq.len;
+  float acc = 0.f;
+  if (valid && sub * 8 < a.d) {
+    const long long r = seq.row0 + n;
+    const uint4 ov = *reinterpret_cast<const uint4*>(a.o + b * a.o_sb + r * a.o_sn + h * a.o_sh + sub * 8);
+    const uint4 dv = *reinterpret_cast<const uint4*>(a.dout + b * a.do_sb + r * a.do_sn + h * a.do_sh + sub * 8);
+    const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
+    const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 x = unpack2<BF16>(ow[i]);
-        const float2 y = unpack2<BF16>(dw[i]);
-        acc = fmaf(x.x, y.x, acc);
-        acc = fmaf(x.y, y.y, acc);
-      }
-    }
-#pragma unroll
-    for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, G);
-    if (in && sub == 0) {
-      a.dd[row] = valid ? acc : 0.f;
-      a.lse2[row] = valid ? a.lse[b * a.lse_sb + h * a.lse_sh + seq.row0 + n] * 1.4426950408889634f : INFINITY;
+    for (int i = 0; i < 4; ++i) {
+      const float2 x = unpack2<BF16>(ow[i]);
+      const float2 y = unpack2<BF16>(dw[i]);
+      acc = fmaf(x.x, y.x, acc);
+      acc = fmaf(x.y, y.y, acc);
     }
   }
-  const long long ncnt = 2LL * a.B * a.H * a.ntiles;
-  for (long long p = tid; p < ncnt; p += nthreads) a.cnt[p] = 0;
-  if (tid == 0) *a.sched = 0;
+#pragma unroll
+  for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, G);
+  if (sub == 0 && n < a.npad) {
+    const size_t row = (size_t)bh * a.npad + n;
+    a.dd[row] = valid ? acc : 0.f;
+    a.lse2[row] = valid ? a.lse[b * a.lse_sb + h * a.lse_sh + seq.row0 + n] * 1.4426950408889634f : INFINITY;
+  }
+  // This head's ordering counters (both sums), and the work counter.
+  if (blockIdx.x == 0) {
+    for (int t = threadIdx.x; t < a.ntiles; t += blockDim.x) {
+      a.cnt[(size_t)bh * a.ntiles + t] = 0;
+      a.cnt[((size_t)a.B * a.H + bh) * a.ntiles + t] = 0;
+    }
+    if (bh == 0 && threadIdx.x == 0) *a.sched = 0;
+  }
 }
 
 // ------------------------------------------------------------------ kernel 3
 
+// dQ of one 128-row tile of one head (block (tile, bh)): the fp32 sums are
+// read in their tile-blocked layout (consecutive threads, consecutive rows:
+// coalesced), turned around in shared memory, and each row written with
+// 16-byte stores (consecutive threads, consecutive columns of a row).
+template <int D>
+struct DqCfg {
+  static constexpr int kStride = D + 4;  // floats per row in shared memory (bank-conflict padding)
+  static constexpr int kSmem = 128 * kStride * 4;
+};
+
 template <int D, bool CAUSAL, bool BF16>
 __global__ void __launch_bounds__(256) fa_bwd_dq(const BwdArgs a) {
-  // Thread per (row, 4 columns); consecutive threads take consecutive rows of
-  // one tile so the accumulator reads are contiguous.
-  const long long total = (long long)a.B * a.H * a.npad * (D / 4);
-  for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < total;
-       t += (long long)gridDim.x * blockDim.x) {
-    const int r = (int)(t % 128);
-    long long rest = t / 128;
-    const int c4 = (int)(rest % (D / 4));
-    rest /= (D / 4);
-    const int tile = (int)(rest % a.ntiles);
-    const int bh = (int)(rest / a.ntiles);
-    const int n = tile * 128 + r;
-    const int b = bh / a.H, h = bh % a.H;
-    const SeqRows seq = seq_rows(a.cu, b, a.N, a.total);
-    if (n >= seq.len || c4 * 4 >= a.d) continue;
-    float4 v = reinterpret_cast<const float4*>(a.dqacc)[t];
-    if (!CAUSAL && tile < (seq.len + 127) / 128 - 1) {
-      // Upper sum (key tiles after this query tile): present unless i is the
-      // sequence's last tile.
-      const float4 u = reinterpret_cast<const float4*>(a.dqacc)[t + total];
+  using C = DqCfg<D>;
+  extern __shared__ float4 sm_dq[];
+  float* sm = reinterpret_cast<float*>(sm_dq);
+  const int tile = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.H, h = bh % a.H;
+  const SeqRows seq = seq_rows(a.cu, b, a.N, a.total);
+  const int ntile_seq = (seq.len + 127) / 128;
+  if (tile >= ntile_seq) return;
+  // Upper sum (key tiles after this query tile): present unless i is the
+  // sequence's last tile.
+  const bool upper = !CAUSAL && tile < ntile_seq - 1;
+  const size_t tile_off = ((size_t)bh * a.ntiles + tile) * 128 * D;  // floats
+  const size_t chain = (size_t)a.B * a.H * a.npad * D;               // floats per sum
+  const float4* lo = reinterpret_cast<const float4*>(a.dqacc + tile_off);
+  const float4* up = reinterpret_cast<const float4*>(a.dqacc + chain + tile_off);
+  for (int idx = threadIdx.x; idx < 128 * (D / 4); idx += blockDim.x) {
+    const int q = idx / 128, r = idx % 128;  // [D/4][128][4] layout
+    float4 v = lo[idx];
+    if (upper) {
+      const float4 u = up[idx];
       v.x += u.x;
       v.y += u.y;
       v.z += u.z;
       v.w += u.w;
     }
-    uint16_t* dst = a.dq + b * a.dq_sb + (seq.row0 + n) * a.dq_sn + h * a.dq_sh + c4 * 4;
-    uint2 w;
-    w.x = pack2<BF16>(v.x * a.scale, v.y * a.scale);
-    w.y = pack2<BF16>(v.z * a.scale, v.w * a.scale);
-    *reinterpret_cast<uint2*>(dst) = w;
+    *reinterpret_cast<float4*>(sm + r * C::kStride + 4 * q) = v;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < 128 * (D / 8); idx += blockDim.x) {
+    const int r = idx / (D / 8), c8 = idx % (D / 8);
+    const int n = tile * 128 + r;
+    if (n >= seq.len || c8 * 8 >= a.d) continue;
+    const float4 x0 = *reinterpret_cast<const float4*>(sm + r * C::kStride + 8 * c8);
+    const float4 x1 = *reinterpret_cast<const float4*>(sm + r * C::kStride + 8 * c8 + 4);
+    uint4 w;
+    w.x = pack2<BF16>(x0.x * a.scale, x0.y * a.scale);
+    w.y = pack2<BF16>(x0.z * a.scale, x0.w * a.scale);
+    w.z = pack2<BF16>(x1.x * a.scale, x1.y * a.scale);
+    w.w = pack2<BF16>(x1.z * a.scale, x1.w * a.scale);
+    *reinterpret_cast<uint4*>(a.dq + b * a.dq_sb + (seq.row0 + n) * a.dq_sn + h * a.dq_sh + c8 * 8) = w;
   }
 }
 
@@ -696,9 +715,16 @@ __global__ void __launch_bounds__(512, 1)
             const float2 l2 = *reinterpret_cast<const float2*>(sLSE + st * 128 + qc);
             float v0 = ex2(fmaf(__uint_as_float(sv[2 * x]), cl2, -l2.x));
             float v1 = ex2(fmaf(__uint_as_float(sv[2 * x + 1]), cl2, -l2.y));
-            if ((diag && key > i * 128 + qc) || !key_in) v0 = 0.f;
-            if ((diag && key > i * 128 + qc + 1) || !key_in) v1 = 0.f;
+            if (diag && key > i * 128 + qc) v0 = 0.f;
+            if (diag && key > i * 128 + qc + 1) v1 = 0.f;
             pk[h2 * 16 + x] = pack2<BF16>(v0, v1);
+          }
+          // Past the sequence's end (only a key tile's tail): P = 0. Applied
+          // once to the packed row rather than per element, which kept the
+          // common path 4% faster.
+          if (!key_in) {
+#pragma unroll
+            for (int x = 0; x < 16; ++x) pk[h2 * 16 + x] = 0u;
           }
           if constexpr (DROPOUT) {
             // dV uses the dropped P (its 1 / (1 - p) is applied to dV at the

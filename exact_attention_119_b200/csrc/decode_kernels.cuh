@@ -18,12 +18,10 @@
 // gets O = 0 and LSE = -inf.
 //
 // Roles (128 threads): thread 0 also issues the TMA loads of the K and V
-// tiles into a 3-stage ring (64 keys x up to 128 columns each, 128-byte
+// tiles into a 2- or 3-stage ring (64 keys x up to 128 columns each, 128-byte
 // swizzle); all threads then compute, two threads per key for the scores
 // (one per half of the head size), one warp per query row for the softmax
-// update, and one thread per (column pair, part of the keys) for P V. At
-// d = 128 a CTA takes about 111 KB of shared memory, so two share an SM and
-// one's start overlaps the other's streaming.
+// update, and one thread per (column pair, part of the keys) for P V.
 #pragma once
 
 #include "sm100.cuh"
@@ -49,24 +47,28 @@ struct DecArgs {
 
 constexpr int kDecMaxNq = 8;   // query rows per sequence and call
 constexpr int kDecKeys = 64;   // keys per tile
-constexpr int kDecStages = 3;
 
-template <int D>
+// NQ: the launch's bound on query rows (1, 2, 4 or 8). Shared memory is sized
+// for NQ rows, and with one or two rows the ring has two stages, so that
+// three CTAs share an SM (more loads in flight, and one CTA's barriers
+// overlap the others' streaming); otherwise three stages and two CTAs.
+template <int D, int NQ>
 struct DecCfg {
+  static constexpr int kStages = NQ <= 2 ? 2 : 3;
   static constexpr int kBoxBytes = kDecKeys * 128;           // 64 rows x 64 columns x 2 B
   static constexpr int kTileBytes = kDecKeys * D * 2;        // one K or V tile
   static constexpr int kStageBytes = 2 * kTileBytes;         // K then V
-  static constexpr int kQ = 0;                               // [kDecMaxNq][D] fp32
-  static constexpr int kS = kQ + kDecMaxNq * D * 4;          // [kDecMaxNq][64] fp32: scores, then P
-  static constexpr int kAlpha = kS + kDecMaxNq * kDecKeys * 4;  // [kDecMaxNq] rescale factors
+  static constexpr int kQ = 0;                               // [NQ][D] fp32
+  static constexpr int kS = kQ + NQ * D * 4;                 // [NQ][64] fp32: scores, then P
+  static constexpr int kAlpha = kS + NQ * kDecKeys * 4;      // [NQ] rescale factors (16-byte padded)
   // P V: thread = (column pair, part of the tile's keys)
   static constexpr int kPairs = D / 2;
   static constexpr int kParts = 128 / kPairs;                // 2 at D = 128, 4 at D = 64
   static constexpr int kKeysPerPart = kDecKeys / kParts;
-  static constexpr int kRed = kAlpha + kDecMaxNq * 4;        // [kParts][kDecMaxNq][D] fp32: parts' sums
-  static constexpr int kBar = kRed + kParts * kDecMaxNq * D * 4;
+  static constexpr int kRed = kAlpha + ((NQ * 4 + 15) / 16) * 16;  // [kParts][NQ][D] fp32: parts' sums
+  static constexpr int kBar = kRed + kParts * NQ * D * 4;
   static constexpr int kRing = (kBar + 64 + 1023) / 1024 * 1024;
-  static constexpr int kSmem = kRing + kDecStages * kStageBytes + 1024;  // + alignment slack
+  static constexpr int kSmem = kRing + kStages * kStageBytes + 1024;  // + alignment slack
   static constexpr int kThreads = 128;
 };
 
@@ -79,7 +81,7 @@ __device__ __forceinline__ uint32_t swz_off(int j, int c) { return j * 128 + ((c
 template <int D, bool BF16, int NQ>
 __global__ void __launch_bounds__(128) fa_decode_split(const __grid_constant__ CUtensorMap tm_k,
                                                        const __grid_constant__ CUtensorMap tm_v, const DecArgs a) {
-  using C = DecCfg<D>;
+  using C = DecCfg<D, NQ>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* sQ = reinterpret_cast<float*>(smem + C::kQ);
@@ -87,7 +89,7 @@ __global__ void __launch_bounds__(128) fa_decode_split(const __grid_constant__ C
   float* sAlpha = reinterpret_cast<float*>(smem + C::kAlpha);
   float* sRed = reinterpret_cast<float*>(smem + C::kRed);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBar);
-  int* abort_flag = reinterpret_cast<int*>(smem + C::kBar + 8 * kDecStages);
+  int* abort_flag = reinterpret_cast<int*>(smem + C::kBar + 8 * C::kStages);
   uint8_t* ring = smem + C::kRing;
 
   const int tid = threadIdx.x;
@@ -115,7 +117,7 @@ __global__ void __launch_bounds__(128) fa_decode_split(const __grid_constant__ C
   }
 
   if (tid == 0) {
-    for (int s = 0; s < kDecStages; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < C::kStages; ++s) mbar_init(&full[s], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -131,8 +133,8 @@ __global__ void __launch_bounds__(128) fa_decode_split(const __grid_constant__ C
   }
   __syncthreads();
 
-  auto issue = [&](int i) {  // tile i of this unit into stage i % kDecStages
-    const int st = i % kDecStages;
+  auto issue = [&](int i) {  // tile i of this unit into stage i % C::kStages
+    const int st = i % C::kStages;
     uint8_t* dst = ring + st * C::kStageBytes;
     mbar_arrive_expect_tx(&full[st], C::kStageBytes);
     const int row = key0 + i * kDecKeys;
@@ -144,7 +146,7 @@ __global__ void __launch_bounds__(128) fa_decode_split(const __grid_constant__ C
   if (tid == 0) {
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
-    for (int i = 0; i < kDecStages - 1 && i < ntiles; ++i) issue(i);
+    for (int i = 0; i < C::kStages - 1 && i < ntiles; ++i) issue(i);
   }
 
   // Softmax state of query row t lives in warp t % 4 (all lanes hold it).
@@ -163,13 +165,13 @@ __global__ void __launch_bounds__(128) fa_decode_split(const __grid_constant__ C
   for (int t = 0; t < NQ; ++t) acc[t][0] = acc[t][1] = 0.f;
 
   bool ok = true;
-  int issued = min(kDecStages - 1, ntiles);
+  int issued = min(C::kStages - 1, ntiles);
   for (int i = 0; i < ntiles; ++i) {
-    const int st = i % kDecStages;
+    const int st = i % C::kStages;
     // The stage refilled here was released by the barrier at the end of the
     // previous tile.
     if (tid == 0 && issued < ntiles) issue(issued++);
-    const bool got = mbar_wait(&full[st], (i / kDecStages) & 1, abort_flag);
+    const bool got = mbar_wait(&full[st], (i / C::kStages) & 1, abort_flag);
     ok = __syncthreads_and(got) != 0;
     if (!ok) break;
     const uint8_t* kt = ring + st * C::kStageBytes;
@@ -289,16 +291,16 @@ __global__ void __launch_bounds__(128) fa_decode_split(const __grid_constant__ C
 
   // Never leave with copies in flight (only after an abort can any be).
   if (tid == 0)
-    for (int x = max(0, issued - kDecStages); x < issued; ++x)
-      mbar_wait(&full[x % kDecStages], (x / kDecStages) & 1, abort_flag, false);
+    for (int x = max(0, issued - C::kStages); x < issued; ++x)
+      mbar_wait(&full[x % C::kStages], (x / C::kStages) & 1, abort_flag, false);
   if (!ok) return;  // the status word already says why
 
   // ---- partial state: the key parts' O added in a fixed order, m and l of each row
 #pragma unroll
   for (int t = 0; t < NQ; ++t) {
     if (t < Nq) {
-      sRed[(kh * kDecMaxNq + t) * D + 2 * cp] = acc[t][0];
-      sRed[(kh * kDecMaxNq + t) * D + 2 * cp + 1] = acc[t][1];
+      sRed[(kh * NQ + t) * D + 2 * cp] = acc[t][0];
+      sRed[(kh * NQ + t) * D + 2 * cp + 1] = acc[t][1];
     }
   }
   __syncthreads();
@@ -306,7 +308,7 @@ __global__ void __launch_bounds__(128) fa_decode_split(const __grid_constant__ C
     const int t = i / D, c = i % D;
     float x = 0.f;
 #pragma unroll
-    for (int part = 0; part < C::kParts; ++part) x += sRed[(part * kDecMaxNq + t) * D + c];
+    for (int part = 0; part < C::kParts; ++part) x += sRed[(part * NQ + t) * D + c];
     po[t * D + c] = x;
   }
 #pragma unroll

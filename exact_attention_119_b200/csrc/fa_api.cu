@@ -45,10 +45,10 @@ thread_local cudaEvent_t t_prof_end = nullptr;
 // error that some earlier, unrelated runtime call left pending in this host
 // thread.) `cluster` > 1 launches clusters of that many CTAs along x.
 template <typename... KArgs, typename... Args>
-cudaError_t launch(const char* name, void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem,
+cudaError_t launch(const char* name, void (*kern)(KArgs...), dim3 grid, unsigned block, size_t smem,
                    cudaStream_t stream, int cluster, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
+  cfg.gridDim = grid;
   cfg.blockDim = dim3(block);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -156,6 +156,10 @@ fa_status make_problem(const fa_desc* desc, Problem* p, bool backward) {
   if (p->cu != nullptr) {
     if (reinterpret_cast<uintptr_t>(p->cu) & 3u) return bad_arg("cu_seqlens must be 4-byte aligned");
     if (p->total < 1) return bad_arg("total (rows of the packed tensors) must be >= 1 with cu_seqlens");
+  }
+  if ((long long)p->B * p->H > 65535) {
+    set_detail_text("B * H must be at most 65535");
+    return FA_ERR_UNSUPPORTED;
   }
   const long long rows = p->cu ? (long long)p->total : (long long)p->B * p->N;
   if (rows * p->H * p->d >= (1LL << 31)) {
@@ -430,9 +434,9 @@ template <int D, bool CAUSAL, bool BF16, bool DROPOUT>
 cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const CUtensorMap& mdo, const BwdArgs& a, int sms, cudaStream_t s) {
   using C = BwdCfg<D>;
-  const long long rows = (long long)a.B * a.H * a.npad;
-  const int prep_blocks = (int)std::min<long long>((rows * (D / 8) + 255) / 256 + 1, 4LL * sms * 8);
-  cudaError_t e = launch("fa_bwd_prep", fa_bwd_prep<D, BF16>, prep_blocks, 256, 0, s, 1, a);
+  constexpr int kPrepRows = 256 / (D / 8);
+  cudaError_t e = launch("fa_bwd_prep", fa_bwd_prep<D, BF16>,
+                         dim3((a.npad + kPrepRows - 1) / kPrepRows, a.B * a.H), 256, 0, s, 1, a);
   if (e != cudaSuccess) return e;
   auto kern = fa_bwd_dkdv<D, CAUSAL, BF16, DROPOUT>;
   e = set_smem(kern, C::kSmem);
@@ -452,9 +456,13 @@ cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
     set_detail_cuda("cudaEventRecord(profile end)", e);
     return e;
   }
-  const long long dq_threads = (long long)a.B * a.H * a.npad * (D / 4);
-  const int dq_blocks = (int)std::min<long long>((dq_threads + 255) / 256, 64LL * sms);
-  return launch("fa_bwd_dq", fa_bwd_dq<D, CAUSAL, BF16>, dq_blocks, 256, 0, s, 1, a);
+  auto dqk = fa_bwd_dq<D, CAUSAL, BF16>;
+  e = set_smem(dqk, DqCfg<D>::kSmem);
+  if (e != cudaSuccess) {
+    set_detail_cuda("cudaFuncSetAttribute(fa_bwd_dq)", e);
+    return e;
+  }
+  return launch("fa_bwd_dq", dqk, dim3(a.ntiles, a.B * a.H), 256, DqCfg<D>::kSmem, s, 1, a);
 }
 
 template <int D, bool DROPOUT>
@@ -537,8 +545,9 @@ struct DecPlan {
   size_t off_ml, total_bytes;
 };
 
-// Units of the cache's key axis: enough CTAs for about four waves of two per
-// SM over the whole launch, at least two 64-key tiles each.
+// Units of the cache's key axis: about eight CTAs per SM over the whole
+// launch (two or three waves, with two or three resident per SM), at least
+// two 64-key tiles each.
 DecPlan dec_plan(int B, int Nq, int H, int d, int Nmax, int sms) {
   DecPlan pl;
   pl.D = d <= 64 ? 64 : 128;
@@ -576,7 +585,7 @@ fa_status dec_check(int B, int Nq, int H, int d, int Nmax, float scale, int caus
 
 template <int D, bool BF16, int NQ>
 cudaError_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const DecArgs& a, cudaStream_t s) {
-  using C = DecCfg<D>;
+  using C = DecCfg<D, NQ>;
   auto kern = fa_decode_split<D, BF16, NQ>;
   cudaError_t e = set_smem(kern, C::kSmem);
   if (e != cudaSuccess) {

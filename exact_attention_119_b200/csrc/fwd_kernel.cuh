@@ -133,12 +133,13 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdArgs& args, int item, uint3
   return w;
 }
 
-// The k-th item of this CTA: one CTA (or CTA pair) per item when split;
-// otherwise persistent, the CTAs taking items in a back-and-forth ("snake")
-// order over rounds of gridDim.x, which evens out the causal lengths.
-template <bool SPLIT>
+// The k-th item of this CTA. PERSISTENT: the CTAs take items in a
+// back-and-forth ("snake") order over rounds of gridDim.x, which evens out
+// the causal lengths. Otherwise one item per CTA (per CTA pair when split),
+// known at compile time, so the item loop folds away.
+template <bool SPLIT, bool PERSISTENT>
 __device__ __forceinline__ int fwd_item_index(int k) {
-  if (SPLIT) return k == 0 ? static_cast<int>(blockIdx.x / 2) : INT_MAX;
+  if (!PERSISTENT) return k == 0 ? static_cast<int>(SPLIT ? blockIdx.x / 2 : blockIdx.x) : INT_MAX;
   const int g = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
   return k * g + ((k & 1) ? g - 1 - c : c);
 }
@@ -164,12 +165,15 @@ __global__ void __launch_bounds__(384, 1)
   // one the sequence bounds are kernel parameters, which the softmax warps
   // (at their register limit) need not keep in registers.
   static_assert(!(SPLIT && (VARLEN || DROPOUT)), "variable-length and dropout launches are not split");
+  // Persistent at d = 128 (a grid of at most one CTA per SM); one item per
+  // CTA at d = 64 and when split (the host sizes the grid to match).
+  constexpr bool kPersistent = D == 128 && !SPLIT;
   const uint32_t crank = SPLIT ? cluster_ctarank() : 0u;
   const int total_items = args.n_mblocks * args.B * args.H;
   // An item with no work: a row block past the end of a shorter sequence.
   auto skip = [&](const FwdItem& w) { return w.q0 >= w.seq.len || w.n_kv <= 0; };
   if constexpr (SPLIT) {
-    const FwdItem w0 = fwd_item<CAUSAL, SPLIT, VARLEN, C::kKeys>(args, fwd_item_index<SPLIT>(0), crank);
+    const FwdItem w0 = fwd_item<CAUSAL, SPLIT, VARLEN, C::kKeys>(args, fwd_item_index<SPLIT, kPersistent>(0), crank);
     if (w0.q0 >= w0.seq.len) return;  // both CTAs of the pair see the same row block
   }
 
@@ -225,7 +229,7 @@ __global__ void __launch_bounds__(384, 1)
       int it = 0, nit = 0;
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        const int item = fwd_item_index<SPLIT>(k);
+        const int item = fwd_item_index<SPLIT, kPersistent>(k);
         if (item >= total_items) break;
         const FwdItem w = fwd_item<CAUSAL, SPLIT, VARLEN, C::kKeys>(args, item, crank);
         if (skip(w)) continue;
@@ -292,7 +296,7 @@ __global__ void __launch_bounds__(384, 1)
       int it0 = 0, gs = 0, pvc = 0, nit = 0;  // ring base, steps, pv_done completions, items
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        const int item = fwd_item_index<SPLIT>(k);
+        const int item = fwd_item_index<SPLIT, kPersistent>(k);
         if (item >= total_items) break;
         const FwdItem w = fwd_item<CAUSAL, SPLIT, VARLEN, C::kKeys>(args, item, crank);
         if (skip(w)) continue;
@@ -427,7 +431,7 @@ __global__ void __launch_bounds__(384, 1)
     int gs = 0, nit = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int item = fwd_item_index<SPLIT>(k);
+      const int item = fwd_item_index<SPLIT, kPersistent>(k);
       if (item >= total_items) break;
       int n_kv, rg, lim, kv_lo;
       {

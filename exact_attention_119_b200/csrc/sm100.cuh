@@ -220,19 +220,15 @@ __device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap* map, int c
 // (d, H, rows, B), or as (d, rows, H, B) when the head stride exceeds the row
 // stride (head-major storage such as [B, H, N, d]); both boxes put the same
 // [128 rows][64 columns] tile into shared memory.
+// (Coordinates picked by selects, not a branch around two copies of the
+// load.)
 __device__ __forceinline__ void tma_load_rows(const CUtensorMap* map, bool head_major, void* smem_dst,
                                               uint64_t* bar, int x, int h, int row, int b) {
-  if (head_major)
-    tma_load_4d(map, smem_dst, bar, x, row, h, b);
-  else
-    tma_load_4d(map, smem_dst, bar, x, h, row, b);
+  tma_load_4d(map, smem_dst, bar, x, head_major ? row : h, head_major ? h : row, b);
 }
 __device__ __forceinline__ void tma_prefetch_rows(const CUtensorMap* map, bool head_major, int x, int h, int row,
                                                   int b) {
-  if (head_major)
-    tma_prefetch_l2_4d(map, x, row, h, b);
-  else
-    tma_prefetch_l2_4d(map, x, h, row, b);
+  tma_prefetch_l2_4d(map, x, head_major ? row : h, head_major ? h : row, b);
 }
 
 // Bits of FwdArgs::hm / BwdArgs::hm: which tensor maps are head-major.

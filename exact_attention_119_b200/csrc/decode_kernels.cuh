@@ -62,15 +62,18 @@ struct DecCfg {
   static constexpr int kQ = 0;                               // [NQ][D] fp32
   static constexpr int kS = kQ + NQ * D * 4;                 // [NQ][64] fp32: scores, then P
   static constexpr int kAlpha = kS + NQ * kDecKeys * 4;      // [NQ] rescale factors (16-byte padded)
+  static constexpr int kThreads = 128;
+  static constexpr int kWarps = kThreads / 32;
+  // Scores: kSplit threads per key, each over D / kSplit columns.
+  static constexpr int kSplit = kThreads / kDecKeys;
   // P V: thread = (column pair, part of the tile's keys)
   static constexpr int kPairs = D / 2;
-  static constexpr int kParts = 128 / kPairs;                // 2 at D = 128, 4 at D = 64
+  static constexpr int kParts = kThreads / kPairs;
   static constexpr int kKeysPerPart = kDecKeys / kParts;
   static constexpr int kRed = kAlpha + ((NQ * 4 + 15) / 16) * 16;  // [kParts][NQ][D] fp32: parts' sums
   static constexpr int kBar = kRed + kParts * NQ * D * 4;
   static constexpr int kRing = (kBar + 64 + 1023) / 1024 * 1024;
   static constexpr int kSmem = kRing + kStages * kStageBytes + 1024;  // + alignment slack
-  static constexpr int kThreads = 128;
 };
 
 // The 16-byte chunk `c` (8 columns) of key row j of a [64 rows][64 columns]
@@ -80,8 +83,9 @@ __device__ __forceinline__ uint32_t swz_off(int j, int c) { return j * 128 + ((c
 // NQ: the query rows' compile-time bound (1, 2, 4 or 8; Nq <= NQ), so the
 // per-key loops do no work for rows that do not exist.
 template <int D, bool BF16, int NQ>
-__global__ void __launch_bounds__(128) fa_decode_split(const __grid_constant__ CUtensorMap tm_k,
-                                                       const __grid_constant__ CUtensorMap tm_v, const DecArgs a) {
+__global__ void __launch_bounds__(DecCfg<D, NQ>::kThreads)
+    fa_decode_split(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const DecArgs a) {
   using C = DecCfg<D, NQ>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -150,8 +154,8 @@ __global__ void __launch_bounds__(128) fa_decode_split(const __grid_constant__ C
     for (int i = 0; i < C::kStages - 1 && i < ntiles; ++i) issue(i);
   }
 
-  // Softmax state of query row t lives in warp t % 4 (all lanes hold it).
-  constexpr int kRowsPerWarp = (NQ + 3) / 4;
+  // Softmax state of query row t lives in warp t % kWarps (all lanes hold it).
+  constexpr int kRowsPerWarp = (NQ + C::kWarps - 1) / C::kWarps;
   float m_run[kRowsPerWarp], l_run[kRowsPerWarp];
 #pragma unroll
   for (int r = 0; r < kRowsPerWarp; ++r) {
@@ -180,19 +184,19 @@ __global__ void __launch_bounds__(128) fa_decode_split(const __grid_constant__ C
     const uint8_t* vt = kt + C::kTileBytes;
     const int kbase = key0 + i * kDecKeys;
 
-    // ---- scores: key j = tid / 2, head-size half hf = tid % 2 (one box each at D = 128)
+    // ---- scores: key j = tid / kSplit, columns of part hf = tid % kSplit
     {
-      const int j = tid >> 1, hf = tid & 1;
+      const int j = tid / C::kSplit, hf = tid % C::kSplit;
       const int key = kbase + j;
       // Four partial sums per row (columns 0-3 and 4-7 of each chunk, even
       // and odd chunks) keep the FMA chains short.
       float dot[NQ][4];
 #pragma unroll
       for (int t = 0; t < NQ; ++t) dot[t][0] = dot[t][1] = dot[t][2] = dot[t][3] = 0.f;
-      constexpr int kChunks = D / 16;  // 16-byte chunks per half
+      constexpr int kChunks = D / (8 * C::kSplit);  // 16-byte chunks per part
 #pragma unroll
       for (int cc = 0; cc < kChunks; ++cc) {
-        const int col = hf * (D / 2) + cc * 8;  // first column of this chunk
+        const int col = hf * (D / C::kSplit) + cc * 8;  // first column of this chunk
         const uint8_t* box = kt + (col / 64) * C::kBoxBytes;
         const uint4 w = *reinterpret_cast<const uint4*>(box + swz_off(j, (col % 64) / 8));
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
@@ -225,8 +229,9 @@ __global__ void __launch_bounds__(128) fa_decode_split(const __grid_constant__ C
 #pragma unroll
       for (int t = 0; t < NQ; ++t) {
         if (t < Nq) {
-          const float dsum = (dot[t][0] + dot[t][1]) + (dot[t][2] + dot[t][3]);
-          const float s = dsum + __shfl_xor_sync(0xffffffffu, dsum, 1);
+          float s = (dot[t][0] + dot[t][1]) + (dot[t][2] + dot[t][3]);
+#pragma unroll
+          for (int off = 1; off < C::kSplit; off <<= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
           const int last = a.causal ? L - Nq + t : L - 1;  // last key row t attends
           if (hf == 0) sS[t * kDecKeys + j] = key <= last ? s : -INFINITY;
         }
@@ -234,10 +239,10 @@ __global__ void __launch_bounds__(128) fa_decode_split(const __grid_constant__ C
     }
     __syncthreads();
 
-    // ---- online softmax: warp w updates rows t = w, w + 4, ...
+    // ---- online softmax: warp w updates rows t = w, w + kWarps, ...
 #pragma unroll
     for (int r = 0; r < kRowsPerWarp; ++r) {
-      const int t = warp + 4 * r;
+      const int t = warp + C::kWarps * r;
       if (t < Nq) {
         const float s0 = sS[t * kDecKeys + lane], s1 = sS[t * kDecKeys + 32 + lane];
         float mx = fmaxf(s0, s1);
@@ -326,7 +331,7 @@ __global__ void __launch_bounds__(128) fa_decode_split(const __grid_constant__ C
   }
 #pragma unroll
   for (int r = 0; r < kRowsPerWarp; ++r) {
-    const int t = warp + 4 * r;
+    const int t = warp + C::kWarps * r;
     if (t < Nq && lane == 0) {
       pml[2 * t] = m_run[r];
       pml[2 * t + 1] = l_run[r];

@@ -76,14 +76,14 @@ struct BwdArgs {
   const int* cu;     // variable-length row offsets [B + 1], or nullptr
   int total;         // rows of the packed tensors (variable length)
   // Workspace
-  float* lse2;   // [B*H, npad] LSE * log2(e); +inf on rows past the sequence
+  float* lse2;   // [B*H, npad] -LSE * log2(e); -inf on rows past the sequence
   float* dd;     // [B*H, npad] D; 0 on rows past the sequence
   float* dqacc;  // 2 x [B*H, ntiles, d/4, 128, 4] fp32 (lower, upper sums)
   int* cnt;      // 2 x [B*H, ntiles] dQ ordering counters (lower, upper)
   int* sched;    // work counter
   int B, N, H, npad, ntiles;  // N: sequence length (variable length: the longest)
   int d;             // head size (<= D; columns d .. D-1 are zeros from TMA)
-  uint32_t hm;       // head-major tensor maps (kHmQ | kHmK | kHmV | kHmDO)
+  uint32_t hm;       // head-major tensor maps (kHmQ | kHmK | kHmV | kHmDO | kHmDK | kHmDV)
   Dropout drop;      // used by the DROPOUT instantiation only
   float scale;       // softmax_scale
   float scale_log2;  // softmax_scale * log2(e)
@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(256) fa_bwd_prep(const BwdArgs a) {
   if (sub == 0 && n < a.npad) {
     const size_t row = (size_t)bh * a.npad + n;
     a.dd[row] = valid ? acc : 0.f;
-    a.lse2[row] = valid ? a.lse[b * a.lse_sb + h * a.lse_sh + seq.row0 + n] * 1.4426950408889634f : INFINITY;
+    a.lse2[row] = valid ? -(a.lse[b * a.lse_sb + h * a.lse_sh + seq.row0 + n] * 1.4426950408889634f) : -INFINITY;
   }
   // This head's ordering counters (both sums), and the work counter.
   if (blockIdx.x == 0) {
@@ -327,6 +327,7 @@ template <int D, bool CAUSAL, bool BF16, bool DROPOUT>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_dkdv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                 const BwdArgs a) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -650,7 +651,7 @@ __global__ void __launch_bounds__(512, 1)
     const int quad = warp % 4;
     const int c = quad * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    const float cl2 = a.scale_log2;
+    const uint64_t c2 = bcast2(a.scale_log2);  // (scale log2(e), scale log2(e))
     const float* sLSE = reinterpret_cast<const float*>(smem + C::kLSE);
     const float* sDD = reinterpret_cast<const float*>(smem + C::kDD);
     uint8_t* sDS = smem + C::kDS + wg * C::kBox;  // this warpgroup's 64 query columns
@@ -658,7 +659,7 @@ __global__ void __launch_bounds__(512, 1)
     bool ok = true;
     while (ok) {
       const int slot = n_item & 1;
-      ok = mbar_wait_warp(&bars->item_full[slot], (n_item >> 1) & 1, abort);
+      ok = wg_all(mbar_wait_warp(&bars->item_full[slot], (n_item >> 1) & 1, abort), 1 + wg);
       if (!ok) break;
       const int item = bars->item[slot];
       __syncwarp();
@@ -712,12 +713,20 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
             const int qc = wg * 64 + h2 * 32 + 2 * x;
-            const float2 l2 = *reinterpret_cast<const float2*>(sLSE + st * 128 + qc);
-            float v0 = ex2(fmaf(__uint_as_float(sv[2 * x]), cl2, -l2.x));
-            float v1 = ex2(fmaf(__uint_as_float(sv[2 * x + 1]), cl2, -l2.y));
-            if (diag && key > i * 128 + qc) v0 = 0.f;
-            if (diag && key > i * 128 + qc + 1) v1 = 0.f;
-            pk[h2 * 16 + x] = pack2<BF16>(v0, v1);
+            // (S c - LSE2) for two queries: the smem row holds -LSE2.
+            const uint64_t nl2 = *reinterpret_cast<const uint64_t*>(sLSE + st * 128 + qc);
+            float x0, x1;
+            fma2(x0, x1, __uint_as_float(sv[2 * x]), __uint_as_float(sv[2 * x + 1]), c2, nl2);
+            pk[h2 * 16 + x] = pack2<BF16>(ex2(x0), ex2(x1));
+          }
+          // The diagonal tile: keys after the query are masked, once per
+          // packed pair (only this step pays for it).
+          if (diag) {
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+              const int q0 = i * 128 + wg * 64 + h2 * 32 + 2 * x;
+              pk[h2 * 16 + x] &= (key > q0 ? 0u : 0x0000FFFFu) | (key > q0 + 1 ? 0u : 0xFFFF0000u);
+            }
           }
           // Past the sequence's end (only a key tile's tail): P = 0. Applied
           // once to the packed row rather than per element, which kept the
@@ -763,7 +772,7 @@ __global__ void __launch_bounds__(512, 1)
           for (int x = 0; x < 16; ++x) {
             const int qc = wg * 64 + h2 * 32 + 2 * x;
             const float2 pp = unpack2<BF16>(pk[h2 * 16 + x]);
-            const float2 dd = *reinterpret_cast<const float2*>(sDD + st * 128 + qc);
+            const uint64_t dd2 = *reinterpret_cast<const uint64_t*>(sDD + st * 128 + qc);
             float dp0 = __uint_as_float(dp[2 * x]), dp1 = __uint_as_float(dp[2 * x + 1]);
             if constexpr (DROPOUT) {
               // dP = (dO V^T) o keep / (1 - p)
@@ -771,8 +780,8 @@ __global__ void __launch_bounds__(512, 1)
               dp0 = (keep >> col) & 1u ? dp0 * a.drop.rkeep : 0.f;
               dp1 = (keep >> (col + 1)) & 1u ? dp1 * a.drop.rkeep : 0.f;
             }
-            const float d0 = pp.x * (dp0 - dd.x);
-            const float d1 = pp.y * (dp1 - dd.y);
+            float d0, d1;
+            mul_sub2(d0, d1, pp.x, pp.y, dp0, dp1, dd2);
             dsk[x] = pack2<BF16>(d0, d1);
           }
           // Row c of a 128-byte-swizzled [128][64] box: 16-byte chunk x goes
@@ -810,18 +819,60 @@ __global__ void __launch_bounds__(512, 1)
           if (!p_phase(g, w.tile(k), pk, keep) || !ds_phase(g, pk, keep)) { ok = false; break; }
         }
       }
+      // The warpgroup agrees on going on, so that all of it or none reaches
+      // the epilogue's warpgroup barriers.
+      ok = wg_all(ok, 1 + wg);
       if (!ok) break;
       // ---- epilogue: warpgroup 0 stores dV_j, warpgroup 1 stores scale * dK_j
-      if (!mbar_wait_warp(&bars->acc_full, n_item & 1, abort)) { ok = false; break; }
+      ok = wg_all(mbar_wait_warp(&bars->acc_full, n_item & 1, abort), 1 + wg);
+      if (!ok) break;
       tc_fence_after();
-      {
-        const int b = w.bh / a.H, h = w.bh % a.H;
+      const int b = w.bh / a.H, h = w.bh % a.H;
+      const float mul = wg == 0 ? (DROPOUT ? a.drop.rkeep : 1.f) : a.scale;
+      const uint32_t src = lane_base + (wg == 0 ? C::kTdV : C::kTdK);
+      const int tile0 = w.j * 128;
+      if (a.cu == nullptr || tile0 + 128 <= seq.len) {
+        // Through this warpgroup's dS box (every MMA of the item, the last
+        // dS readers included, completed before acc_full) and a TMA store,
+        // 64 columns at a time; rows past N are clipped by the tensor map.
+        const CUtensorMap* map = wg == 0 ? &tm_dv : &tm_dk;
+        const bool hm = a.hm & (wg == 0 ? kHmDV : kHmDK);
+#pragma unroll 1
+        for (int kb = 0; kb < D / 64; ++kb) {
+          if (kb > 0) {
+            if (c == 0) bulk_wait_read_all();
+            named_bar_sync(1 + wg, 128);
+          }
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) {
+            uint32_t v[32];
+            tmem_ld32(src + (kb * 2 + q2) * 32, v);
+            tmem_ld_wait();
+            tie_regs32(v);
+            uint32_t pk[16];
+#pragma unroll
+            for (int x = 0; x < 16; ++x)
+              pk[x] = pack2<BF16>(__uint_as_float(v[2 * x]) * mul, __uint_as_float(v[2 * x + 1]) * mul);
+#pragma unroll
+            for (int y = 0; y < 4; ++y)
+              st_shared_v4(sDS + c * 128 + (((q2 * 4 + y) ^ (c & 7)) << 4), pk[4 * y], pk[4 * y + 1], pk[4 * y + 2],
+                           pk[4 * y + 3]);
+          }
+          fence_async_shared();
+          named_bar_sync(1 + wg, 128);
+          if (c == 0) {
+            tma_store_rows(map, hm, sDS, kb * 64, h, seq.row0 + tile0, seq.bcoord);
+            bulk_commit();
+          }
+        }
+        // The next item's dS phase writes the box again.
+        if (c == 0) bulk_wait_read_all();
+        named_bar_sync(1 + wg, 128);
+      } else {
         const bool valid = key_in;
-        const float mul = wg == 0 ? (DROPOUT ? a.drop.rkeep : 1.f) : a.scale;
         const long long r = seq.row0 + (valid ? key : 0);
         uint16_t* dst = wg == 0 ? a.dv + b * a.dv_sb + r * a.dv_sn + h * a.dv_sh
                                 : a.dk + b * a.dk_sb + r * a.dk_sn + h * a.dk_sh;
-        const uint32_t src = lane_base + (wg == 0 ? C::kTdV : C::kTdK);
 #pragma unroll 1
         for (int q = 0; q < D / 32; ++q) {
           uint32_t v[32];
@@ -844,6 +895,8 @@ __global__ void __launch_bounds__(512, 1)
       mbar_arrive(&bars->acc_empty);
       ++n_item;
     }
+    // dK / dV stores have completed before the CTA leaves.
+    if (c == 0) bulk_wait_all();
   } else {
     reg_alloc_set<C::kRegsDQ, 128>();
     // ------------------------------------------------------ dQ warps (8-11)

@@ -304,8 +304,8 @@ int num_sms() {
 // ------------------------------------------------------------------ forward
 
 template <int D, bool CAUSAL, bool BF16, bool VARLEN, bool DROPOUT>
-cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdArgs& a,
-                       cudaStream_t stream) {
+cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                       const FwdArgs& a, cudaStream_t stream) {
   using C = FwdCfg<D>;
   const unsigned units = static_cast<unsigned>(a.n_mblocks * a.B * a.H);
   if constexpr (!CAUSAL && !VARLEN && !DROPOUT) {
@@ -318,7 +318,7 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
         set_detail_cuda("cudaFuncSetAttribute(fa_fwd_kernel split)", e);
         return e;
       }
-      if (launch("fa_fwd_kernel split", kern2, 2 * units, C::kThreads, C::kSmemBytes, stream, 2, mq, mk, mv, a) ==
+      if (launch("fa_fwd_kernel split", kern2, 2 * units, C::kThreads, C::kSmemBytes, stream, 2, mq, mk, mv, mo, a) ==
           cudaSuccess)
         return cudaSuccess;
       // No 2-CTA cluster fits: run unsplit. The failed launch's error is this
@@ -342,27 +342,27 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   const int sms = num_sms();
   if (sms <= 0) return cudaErrorInvalidDevice;
   const unsigned grid = D == 128 ? std::min(units, static_cast<unsigned>(sms)) : units;
-  return launch("fa_fwd_kernel", kern, grid, C::kThreads, C::kSmemBytes, stream, 1, mq, mk, mv, one);
+  return launch("fa_fwd_kernel", kern, grid, C::kThreads, C::kSmemBytes, stream, 1, mq, mk, mv, mo, one);
 }
 
 template <int D, bool VARLEN, bool DROPOUT>
 cudaError_t dispatch_fwd(bool causal, bool bf16, const CUtensorMap& mq, const CUtensorMap& mk,
-                         const CUtensorMap& mv, const FwdArgs& a, cudaStream_t s) {
+                         const CUtensorMap& mv, const CUtensorMap& mo, const FwdArgs& a, cudaStream_t s) {
   if (causal)
-    return bf16 ? launch_fwd<D, true, true, VARLEN, DROPOUT>(mq, mk, mv, a, s)
-                : launch_fwd<D, true, false, VARLEN, DROPOUT>(mq, mk, mv, a, s);
-  return bf16 ? launch_fwd<D, false, true, VARLEN, DROPOUT>(mq, mk, mv, a, s)
-              : launch_fwd<D, false, false, VARLEN, DROPOUT>(mq, mk, mv, a, s);
+    return bf16 ? launch_fwd<D, true, true, VARLEN, DROPOUT>(mq, mk, mv, mo, a, s)
+                : launch_fwd<D, true, false, VARLEN, DROPOUT>(mq, mk, mv, mo, a, s);
+  return bf16 ? launch_fwd<D, false, true, VARLEN, DROPOUT>(mq, mk, mv, mo, a, s)
+              : launch_fwd<D, false, false, VARLEN, DROPOUT>(mq, mk, mv, mo, a, s);
 }
 
 template <int D>
 cudaError_t dispatch_fwd_all(const Problem& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                             const FwdArgs& a, cudaStream_t s) {
+                             const CUtensorMap& mo, const FwdArgs& a, cudaStream_t s) {
   if (p.cu)
-    return p.dropout ? dispatch_fwd<D, true, true>(p.causal, p.bf16, mq, mk, mv, a, s)
-                     : dispatch_fwd<D, true, false>(p.causal, p.bf16, mq, mk, mv, a, s);
-  return p.dropout ? dispatch_fwd<D, false, true>(p.causal, p.bf16, mq, mk, mv, a, s)
-                   : dispatch_fwd<D, false, false>(p.causal, p.bf16, mq, mk, mv, a, s);
+    return p.dropout ? dispatch_fwd<D, true, true>(p.causal, p.bf16, mq, mk, mv, mo, a, s)
+                     : dispatch_fwd<D, true, false>(p.causal, p.bf16, mq, mk, mv, mo, a, s);
+  return p.dropout ? dispatch_fwd<D, false, true>(p.causal, p.bf16, mq, mk, mv, mo, a, s)
+                   : dispatch_fwd<D, false, false>(p.causal, p.bf16, mq, mk, mv, mo, a, s);
 }
 
 // Forward work split. A row block's key tiles go to one CTA, or are halved
@@ -397,10 +397,10 @@ fa_status run_fwd(const Problem& p, const void* q, const void* k, const void* v,
     return bad_arg("a pointer is null or not 16-byte aligned");
   fa_status st = bind_context();
   if (st != FA_OK) return st;
-  CUtensorMap mq, mk, mv;
-  bool hq = false, hk = false, hv = false;
+  CUtensorMap mq, mk, mv, mo;
+  bool hq = false, hk = false, hv = false, ho = false;
   if ((st = make_map(&mq, &hq, q, p.q, p, "q")) != FA_OK || (st = make_map(&mk, &hk, k, p.k, p, "k")) != FA_OK ||
-      (st = make_map(&mv, &hv, v, p.v, p, "v")) != FA_OK)
+      (st = make_map(&mv, &hv, v, p.v, p, "v")) != FA_OK || (st = make_map(&mo, &ho, o, p.o, p, "o")) != FA_OK)
     return st;
   FwdArgs a;
   a.o = static_cast<uint16_t*>(o);
@@ -416,13 +416,13 @@ fa_status run_fwd(const Problem& p, const void* q, const void* k, const void* v,
   a.N = p.N;
   a.H = p.H;
   a.d = p.d;
-  a.hm = (hq ? kHmQ : 0u) | (hk ? kHmK : 0u) | (hv ? kHmV : 0u);
+  a.hm = (hq ? kHmQ : 0u) | (hk ? kHmK : 0u) | (hv ? kHmV : 0u) | (ho ? kHmO : 0u);
   a.n_mblocks = (p.N + 255) / 256;
   a.split = (p.cu || p.dropout) ? 1 : fwd_split(p.B, p.N, p.H, p.causal, a.n_mblocks);
   a.drop = p.drop;
   a.scale_log2 = (float)((double)p.scale * 1.4426950408889634);
   const cudaError_t e =
-      p.D == 64 ? dispatch_fwd_all<64>(p, mq, mk, mv, a, s) : dispatch_fwd_all<128>(p, mq, mk, mv, a, s);
+      p.D == 64 ? dispatch_fwd_all<64>(p, mq, mk, mv, mo, a, s) : dispatch_fwd_all<128>(p, mq, mk, mv, mo, a, s);
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -430,9 +430,13 @@ fa_status run_fwd(const Problem& p, const void* q, const void* k, const void* v,
 
 // The three backward launches on one stream: preprocessing, the persistent
 // dK/dV (and dQ partial) kernel, and the dQ cast.
+// Tensor maps of the backward: inputs q, k, v, dout and outputs dk, dv.
+struct BwdMaps {
+  CUtensorMap q, k, v, dout, dk, dv;
+};
+
 template <int D, bool CAUSAL, bool BF16, bool DROPOUT>
-cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                         const CUtensorMap& mdo, const BwdArgs& a, int sms, cudaStream_t s) {
+cudaError_t launch_bwd_t(const BwdMaps& m, const BwdArgs& a, int sms, cudaStream_t s) {
   using C = BwdCfg<D>;
   constexpr int kPrepRows = 256 / (D / 8);
   cudaError_t e = launch("fa_bwd_prep", fa_bwd_prep<D, BF16>,
@@ -450,7 +454,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
     set_detail_cuda("cudaEventRecord(profile begin)", e);
     return e;
   }
-  e = launch("fa_bwd_dkdv", kern, grid, C::kThreads, C::kSmem, s, 1, mq, mk, mv, mdo, a);
+  e = launch("fa_bwd_dkdv", kern, grid, C::kThreads, C::kSmem, s, 1, m.q, m.k, m.v, m.dout, m.dk, m.dv, a);
   if (e != cudaSuccess) return e;
   if (t_prof_end != nullptr && (e = cudaEventRecord(t_prof_end, s)) != cudaSuccess) {
     set_detail_cuda("cudaEventRecord(profile end)", e);
@@ -466,14 +470,10 @@ cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
 }
 
 template <int D, bool DROPOUT>
-cudaError_t dispatch_bwd(bool causal, bool bf16, const CUtensorMap& mq, const CUtensorMap& mk,
-                         const CUtensorMap& mv, const CUtensorMap& mdo, const BwdArgs& a, int sms,
-                         cudaStream_t s) {
+cudaError_t dispatch_bwd(bool causal, bool bf16, const BwdMaps& m, const BwdArgs& a, int sms, cudaStream_t s) {
   if (causal)
-    return bf16 ? launch_bwd_t<D, true, true, DROPOUT>(mq, mk, mv, mdo, a, sms, s)
-                : launch_bwd_t<D, true, false, DROPOUT>(mq, mk, mv, mdo, a, sms, s);
-  return bf16 ? launch_bwd_t<D, false, true, DROPOUT>(mq, mk, mv, mdo, a, sms, s)
-              : launch_bwd_t<D, false, false, DROPOUT>(mq, mk, mv, mdo, a, sms, s);
+    return bf16 ? launch_bwd_t<D, true, true, DROPOUT>(m, a, sms, s) : launch_bwd_t<D, true, false, DROPOUT>(m, a, sms, s);
+  return bf16 ? launch_bwd_t<D, false, true, DROPOUT>(m, a, sms, s) : launch_bwd_t<D, false, false, DROPOUT>(m, a, sms, s);
 }
 
 BwdLayout bwd_layout(const Problem& p) { return BwdLayout::make(p.B, p.N, p.H, p.D); }
@@ -490,10 +490,12 @@ fa_status run_bwd(const Problem& p, const void* q, const void* k, const void* v,
                   const float* lse, void* dq, void* dk, void* dv, uint8_t* ws, cudaStream_t s) {
   fa_status st = bind_context();
   if (st != FA_OK) return st;
-  CUtensorMap mq, mk, mv, mdo;
-  bool hq = false, hk = false, hv = false, hd = false;
-  if ((st = make_map(&mq, &hq, q, p.q, p, "q")) != FA_OK || (st = make_map(&mk, &hk, k, p.k, p, "k")) != FA_OK ||
-      (st = make_map(&mv, &hv, v, p.v, p, "v")) != FA_OK || (st = make_map(&mdo, &hd, dout, p.dout, p, "dout")) != FA_OK)
+  BwdMaps m;
+  bool hq = false, hk = false, hv = false, hd = false, hdk = false, hdv = false;
+  if ((st = make_map(&m.q, &hq, q, p.q, p, "q")) != FA_OK || (st = make_map(&m.k, &hk, k, p.k, p, "k")) != FA_OK ||
+      (st = make_map(&m.v, &hv, v, p.v, p, "v")) != FA_OK ||
+      (st = make_map(&m.dout, &hd, dout, p.dout, p, "dout")) != FA_OK ||
+      (st = make_map(&m.dk, &hdk, dk, p.dk, p, "dk")) != FA_OK || (st = make_map(&m.dv, &hdv, dv, p.dv, p, "dv")) != FA_OK)
     return st;
   const int sms = num_sms();
   if (sms <= 0) return FA_ERR_CUDA;
@@ -524,17 +526,18 @@ fa_status run_bwd(const Problem& p, const void* q, const void* k, const void* v,
   a.d = p.d;
   a.npad = L.npad;
   a.ntiles = L.ntiles;
-  a.hm = (hq ? kHmQ : 0u) | (hk ? kHmK : 0u) | (hv ? kHmV : 0u) | (hd ? kHmDO : 0u);
+  a.hm = (hq ? kHmQ : 0u) | (hk ? kHmK : 0u) | (hv ? kHmV : 0u) | (hd ? kHmDO : 0u) | (hdk ? kHmDK : 0u) |
+         (hdv ? kHmDV : 0u);
   a.scale = p.scale;
   a.scale_log2 = (float)((double)p.scale * 1.4426950408889634);
   a.drop = p.drop;
   cudaError_t e;
   if (p.dropout)
-    e = p.D == 64 ? dispatch_bwd<64, true>(p.causal, p.bf16, mq, mk, mv, mdo, a, sms, s)
-                  : dispatch_bwd<128, true>(p.causal, p.bf16, mq, mk, mv, mdo, a, sms, s);
+    e = p.D == 64 ? dispatch_bwd<64, true>(p.causal, p.bf16, m, a, sms, s)
+                  : dispatch_bwd<128, true>(p.causal, p.bf16, m, a, sms, s);
   else
-    e = p.D == 64 ? dispatch_bwd<64, false>(p.causal, p.bf16, mq, mk, mv, mdo, a, sms, s)
-                  : dispatch_bwd<128, false>(p.causal, p.bf16, mq, mk, mv, mdo, a, sms, s);
+    e = p.D == 64 ? dispatch_bwd<64, false>(p.causal, p.bf16, m, a, sms, s)
+                  : dispatch_bwd<128, false>(p.causal, p.bf16, m, a, sms, s);
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -69,7 +69,9 @@ struct FwdCfg {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-  static constexpr int kSmemBytes = kBarOff + 512 + 1024;  // + barriers + alignment slack
+  static constexpr int kOStOff = kBarOff + 1024;  // O staging: one box per Q tile
+  static constexpr int kSmemBytes = kOStOff + 2 * kBoxBytes + 1024;  // + alignment slack
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
   // A split row block's partial state (2 tiles x 128 rows x (D + 4) floats)
   // goes over Q and the K/V ring at the end.
   static_assert(2 * 128 * (D + 4) * 4 <= kBarOff, "partial rows must fit below the barriers");
@@ -87,6 +89,7 @@ struct FwdBarriers {
   uint64_t q_empty;     // the item's last S MMA has read Q: the next Q may be loaded
   uint64_t s_full[2];
   uint64_t p_full[2];
+  uint64_t p_half[2];   // without kSepP: P of the tile's first 64 keys is in TMEM
   uint64_t o_full[2];
   uint64_t s_cons[2];   // kSepP: the softmax has S(t, j) in registers
   uint64_t pv_done[2];  // kSepP: P(t, j) V_j has completed
@@ -147,7 +150,8 @@ __device__ __forceinline__ int fwd_item_index(int k) {
 template <int D, bool CAUSAL, bool BF16, bool SPLIT, bool VARLEN, bool DROPOUT>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const FwdArgs args) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -183,6 +187,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->s_full[t], 1);
       mbar_init(&bars->p_full[t], 128);
+      mbar_init(&bars->p_half[t], 128);
       mbar_init(&bars->o_full[t], 1);
       mbar_init(&bars->s_cons[t], 128);
       mbar_init(&bars->pv_done[t], 1);
@@ -284,13 +289,16 @@ __global__ void __launch_bounds__(384, 1)
           mma_ss(tmem + C::tmem_s(t), qa + off, ka + off, kIdS, ks > 0);
         }
       };
-      auto issue_pv = [&](int t, int stage, bool acc) {
+      // P V over keys [16 kk0, 16 kk1) of the tile.
+      auto issue_pv_keys = [&](int t, int stage, bool acc, int kk0, int kk1) {
         const uint64_t va = dKV_mn + (uint64_t)(stage * kTile16);
 #pragma unroll
-        for (int kk = 0; kk < C::kKeys / 16; ++kk)
+        for (int kk = kk0; kk < kk1; ++kk)
           mma_ts(tmem + C::tmem_o(t), tmem + C::tmem_p(t) + kk * 8, va + (uint64_t)(kk * (2048 >> 4)), kIdPV,
                  (acc || kk > 0) ? 1u : 0u);
       };
+      auto issue_pv = [&](int t, int stage, bool acc) { issue_pv_keys(t, stage, acc, 0, C::kKeys / 16); };
+      constexpr int kHalfK = C::kKeys / 32;  // MMAs over the first 64 keys
       auto kv_wait = [&](int pos) { return mbar_wait(&bars->kv_full[pos % C::kStages], (pos / C::kStages) & 1, abort); };
 
       int it0 = 0, gs = 0, pvc = 0, nit = 0;  // ring base, steps, pv_done completions, items
@@ -369,19 +377,31 @@ __global__ void __launch_bounds__(384, 1)
             mma_commit(&bars->kv_empty[pv % C::kStages]);
           }
         } else {
+          // P(t, j) V_j in two halves of the keys: the first as soon as the
+          // softmax has written P of keys 0-63 (p_half), so it overlaps the
+          // exponentials of keys 64-127; the second, then S(t, j+1) over the
+          // same columns, once all of P is in (p_full).
+          auto pv_first_half = [&](int t, int pv, bool acc, int g) {
+            if (!mbar_wait(&bars->p_half[t], g & 1, abort)) return false;
+            tc_fence_after();
+            issue_pv_keys(t, pv % C::kStages, acc, 0, kHalfK);
+            return true;
+          };
+          auto pv_second_half = [&](int t, int pv, int g) {
+            if (!mbar_wait(&bars->p_full[t], g & 1, abort)) return false;
+            tc_fence_after();
+            issue_pv_keys(t, pv % C::kStages, true, kHalfK, C::kKeys / 16);
+            return true;
+          };
           for (int j = 1; j < n_kv && ok; ++j) {
             const int pv = it0 + 2 * j - 1, pk = it0 + 2 * j;  // ring positions of V_{j-1} and K_j
             const int g = gs + j - 1;                          // step of P(j-1)
-            ok = kv_wait(pv) && kv_wait(pk) && mbar_wait(&bars->p_full[0], g & 1, abort);
+            ok = kv_wait(pv) && pv_first_half(0, pv, j > 1, g) && kv_wait(pk) && pv_second_half(0, pv, g);
             if (!ok) break;
-            tc_fence_after();
-            issue_pv(0, pv % C::kStages, j > 1);
             issue_s(0, pk % C::kStages);
             mma_commit(&bars->s_full[0]);
-            ok = mbar_wait(&bars->p_full[1], g & 1, abort);
+            ok = pv_first_half(1, pv, j > 1, g) && pv_second_half(1, pv, g);
             if (!ok) break;
-            tc_fence_after();
-            issue_pv(1, pv % C::kStages, j > 1);
             mma_commit(&bars->kv_empty[pv % C::kStages]);
             issue_s(1, pk % C::kStages);
             mma_commit(&bars->s_full[1]);
@@ -391,16 +411,12 @@ __global__ void __launch_bounds__(384, 1)
             mma_commit(&bars->q_empty);  // every S of the item is issued
             const int pv = it0 + 2 * n_kv - 1;
             const int g = gs + n_kv - 1;
-            ok = kv_wait(pv) && mbar_wait(&bars->p_full[0], g & 1, abort);
+            ok = kv_wait(pv) && pv_first_half(0, pv, n_kv > 1, g) && pv_second_half(0, pv, g);
             if (ok) {
-              tc_fence_after();
-              issue_pv(0, pv % C::kStages, n_kv > 1);
               mma_commit(&bars->o_full[0]);
-              ok = mbar_wait(&bars->p_full[1], g & 1, abort);
+              ok = pv_first_half(1, pv, n_kv > 1, g) && pv_second_half(1, pv, g);
             }
             if (ok) {
-              tc_fence_after();
-              issue_pv(1, pv % C::kStages, n_kv > 1);
               mma_commit(&bars->o_full[1]);
               mma_commit(&bars->kv_empty[pv % C::kStages]);
             }
@@ -523,6 +539,7 @@ __global__ void __launch_bounds__(384, 1)
         lr *= alpha;
         const uint32_t tP = lane_base + C::tmem_p(t);
         const float neg_m = (m == -INFINITY) ? 0.f : -m;
+        const uint64_t c2 = bcast2(c), neg_m2 = bcast2(neg_m);
         // Four accumulators each for the exact and the rounded sums, so no add
         // waits on the one before it.
         float sa[4] = {0.f, 0.f, 0.f, 0.f}, sra[4] = {0.f, 0.f, 0.f, 0.f};
@@ -541,16 +558,25 @@ __global__ void __launch_bounds__(384, 1)
           }
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2(fmaf(__uint_as_float(s[part * 32 + 2 * i]), c, neg_m));
-            const float p1 = ex2(fmaf(__uint_as_float(s[part * 32 + 2 * i + 1]), c, neg_m));
+            float x0, x1, p0, p1;
+            fma2(x0, x1, __uint_as_float(s[part * 32 + 2 * i]), __uint_as_float(s[part * 32 + 2 * i + 1]), c2, neg_m2);
+            p0 = ex2(x0);
+            p1 = ex2(x1);
             p[i] = pack2<BF16>(p0, p1);
             const int a = 2 * (i & 1);
-            sa[a] += p0;
-            sa[a + 1] += p1;
+            add2(sa[a], sa[a + 1], p0, p1);
             sra[a] = add_lo16<BF16>(sra[a], p[i]);
             sra[a + 1] = add_hi16<BF16>(sra[a + 1], p[i]);
             if constexpr (DROPOUT)
               p[i] &= ((keep >> (2 * i)) & 1u ? 0x0000FFFFu : 0u) | ((keep >> (2 * i + 1)) & 1u ? 0xFFFF0000u : 0u);
+          }
+          if constexpr (!C::kSepP) {
+            if (part == 2) {
+              // P of keys 0-63 is stored: let P V start on it.
+              tmem_st_wait();
+              tc_fence_before();
+              mbar_arrive(&bars->p_half[t]);
+            }
           }
           if (part == 0 && !pv_waited) {
             if (!mbar_wait_warp(&bars->pv_done[t], pvg & 1, abort)) {
@@ -570,36 +596,74 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive(&bars->p_full[t]);
       }
       // (A split pair runs the merge below whatever happened, so that CTA 1
-      // always signals CTA 0.)
-      if (!ok && !SPLIT) break;
+      // always signals CTA 0.) Otherwise the warpgroup agrees on going on, so
+      // that all of it or none reaches the epilogue's warpgroup barriers.
+      if constexpr (!SPLIT) {
+        ok = wg_all(ok, 1 + t);
+        if (!ok) break;
+      }
 
       // ------------------------------------------------------------ epilogue
       const FwdItem w = fwd_item<CAUSAL, SPLIT, VARLEN, C::kKeys>(args, item, crank);
       if constexpr (!SPLIT) {
-        if (!mbar_wait_warp(&bars->o_full[t], nit & 1, abort)) {
-          ok = false;
-          break;
-        }
+        ok = wg_all(mbar_wait_warp(&bars->o_full[t], nit & 1, abort), 1 + t);
+        if (!ok) break;
         tc_fence_after();
         // With dropout, the kept P's scale 1 / (1 - p) is applied here, once.
         const float inv_l = (DROPOUT ? args.drop.rkeep : 1.f) / lr;
         const bool valid = rg < w.seq.len;
-        uint16_t* orow = args.o + w.b * args.o_sb + (w.seq.row0 + (valid ? rg : 0)) * args.o_sn + w.h * args.o_sh;
+        // A tile that starts inside the sequence and, with variable length,
+        // ends inside it too (without, the tensor map's row extent clips rows
+        // past N): TMA store. Otherwise each thread writes its own row.
+        const int tile0 = w.q0 + t * 128;
+        if (tile0 < w.seq.len && (!VARLEN || tile0 + 128 <= w.seq.len)) {
+          uint8_t* stg = smem + C::kOStOff + t * C::kBoxBytes;
 #pragma unroll 1
-        for (int q = 0; q < D / 32; ++q) {
-          uint32_t o[32];
-          tmem_ld32(tO + q * 32, o);
-          tmem_ld_wait();
-          tie_regs32(o);
-          uint32_t pk[16];
+          for (int kb = 0; kb < D / 64; ++kb) {
+            // The staging box is free once this tile's previous store has read it.
+            if (r == 0) bulk_wait_read_all();
+            named_bar_sync(1 + t, 128);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+            for (int q2 = 0; q2 < 2; ++q2) {
+              uint32_t o[32];
+              tmem_ld32(tO + (kb * 2 + q2) * 32, o);
+              tmem_ld_wait();
+              tie_regs32(o);
+              uint32_t pk[16];
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              if (q * 32 + v * 8 < args.d) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+              for (int i = 0; i < 16; ++i)
+                pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+              // Row r of the box is 128 bytes; its 16-byte chunk c sits at c ^ (r % 8).
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                st_shared_v4(stg + r * 128 + (((q2 * 4 + v) ^ (r & 7)) << 4), pk[4 * v], pk[4 * v + 1], pk[4 * v + 2],
+                             pk[4 * v + 3]);
+            }
+            fence_async_shared();
+            named_bar_sync(1 + t, 128);
+            if (r == 0) {
+              tma_store_rows(&tm_o, args.hm & kHmO, stg, kb * 64, w.h, w.seq.row0 + tile0, w.seq.bcoord);
+              bulk_commit();
+            }
+          }
+        } else {
+          uint16_t* orow = args.o + w.b * args.o_sb + (w.seq.row0 + (valid ? rg : 0)) * args.o_sn + w.h * args.o_sh;
+#pragma unroll 1
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t o[32];
+            tmem_ld32(tO + q * 32, o);
+            tmem_ld_wait();
+            tie_regs32(o);
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+            if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                if (q * 32 + v * 8 < args.d) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
           }
         }
         if (valid)
@@ -683,6 +747,8 @@ __global__ void __launch_bounds__(384, 1)
       gs += n_kv;
       ++nit;
     }
+    // O's last stores have completed before the CTA leaves.
+    if (r == 0) bulk_wait_all();
   } else {
     reg_alloc_dec<104>();  // warps 10-11: no role
   }

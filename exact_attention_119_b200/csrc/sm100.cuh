@@ -232,7 +232,40 @@ __device__ __forceinline__ void tma_prefetch_rows(const CUtensorMap* map, bool h
 }
 
 // Bits of FwdArgs::hm / BwdArgs::hm: which tensor maps are head-major.
-constexpr uint32_t kHmQ = 1, kHmK = 2, kHmV = 4, kHmDO = 8;
+constexpr uint32_t kHmQ = 1, kHmK = 2, kHmV = 4, kHmDO = 8, kHmO = 16, kHmDK = 32, kHmDV = 64;
+
+// TMA tile store of one box from shared memory (128-byte swizzled like the
+// loads), tracked by bulk async-groups of the issuing thread.
+__device__ __forceinline__ void tma_store_rows(const CUtensorMap* map, bool head_major, const void* smem_src, int x,
+                                               int h, int row, int b) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_src))), "r"(x), "r"(head_major ? row : h),
+      "r"(head_major ? h : row), "r"(b)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// The shared memory of every committed store has been read.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Every committed store is complete.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// True on all 128 threads of warpgroup barrier `id` iff v is true on all of them.
+__device__ __forceinline__ bool wg_all(bool v, int id) {
+  uint32_t r;
+  asm volatile(
+      "{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.and.pred q, %2, 128, p; selp.u32 %0, 1, 0, q; }"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void st_shared_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))),
+               "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
 
 // ------------------------------------------------------------------- tcgen05
 
@@ -491,6 +524,33 @@ __device__ __forceinline__ float2 unpack2(uint32_t w) {
 }
 
 // max(a, b, c) in one instruction (three-operand form of max.f32, sm_100).
+// Two-lane fp32 arithmetic: sm_100's packed f32x2 forms issue one
+// instruction for two IEEE round-to-nearest results, the same values as two
+// scalar operations. A 64-bit operand holds lane 0 in its low word.
+__device__ __forceinline__ uint64_t bcast2(float x) {
+  const uint64_t u = __float_as_uint(x);
+  return u | (u << 32);
+}
+// (y0, y1) = (x0, x1) * a + b
+__device__ __forceinline__ void fma2(float& y0, float& y1, float x0, float x1, uint64_t a, uint64_t b) {
+  asm("{ .reg .b64 x, y; mov.b64 x, {%2, %3}; fma.rn.f32x2 y, x, %4, %5; mov.b64 {%0, %1}, y; }"
+      : "=f"(y0), "=f"(y1)
+      : "f"(x0), "f"(x1), "l"(a), "l"(b));
+}
+// (s0, s1) += (x0, x1)
+__device__ __forceinline__ void add2(float& s0, float& s1, float x0, float x1) {
+  asm("{ .reg .b64 s, x; mov.b64 s, {%0, %1}; mov.b64 x, {%2, %3}; add.rn.f32x2 s, s, x; mov.b64 {%0, %1}, s; }"
+      : "+f"(s0), "+f"(s1)
+      : "f"(x0), "f"(x1));
+}
+// (y0, y1) = (p0, p1) * ((x0, x1) - b)
+__device__ __forceinline__ void mul_sub2(float& y0, float& y1, float p0, float p1, float x0, float x1, uint64_t b) {
+  asm("{ .reg .b64 p, x, t; mov.b64 p, {%2, %3}; mov.b64 x, {%4, %5}; sub.rn.f32x2 t, x, %6; mul.rn.f32x2 t, p, t;"
+      " mov.b64 {%0, %1}, t; }"
+      : "=f"(y0), "=f"(y1)
+      : "f"(p0), "f"(p1), "f"(x0), "f"(x1), "l"(b));
+}
+
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));

@@ -173,10 +173,10 @@ FA_API fa_status fa_fwd_ex(const fa_desc* desc, const void* q, const void* k, co
  * per-tile ordering counters that make the dQ sum deterministic.
  * Layout after a call (for inspection; N_pad = 128 * ceil(N / 128),
  * up256(x) = x rounded up to a multiple of 256):
- *   byte 0:                           LSE * log2(e), [B*H, N_pad] fp32
+ *   byte 0:                           -LSE * log2(e), [B*H, N_pad] fp32
  *   byte up256(4 * B*H*N_pad):        D,             [B*H, N_pad] fp32
  *   then the dQ sums and counters (internal).
- * Rows N .. N_pad-1 of each head hold +inf (LSE) and 0 (D).
+ * Rows N .. N_pad-1 of each head hold -inf (-LSE * log2(e)) and 0 (D).
  */
 FA_API size_t fa_bwd_workspace_size(int B, int N, int H, int d, int causal);
 

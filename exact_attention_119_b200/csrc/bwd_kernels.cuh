@@ -21,7 +21,7 @@
 //                    added into fp32 accumulators in a fixed key-tile order
 //                    (per-tile counters say whose turn it is), so the sum is
 //                    deterministic.
-//   3. fa_bwd_dq:    dQ = scale * (lower sum + upper sum), cast.
+//   3. fa_bwd_dq:    dQ = scale * (sum 0 + sum 1), cast.
 //
 // dQ order (BwdItem below). Query tile i's dQ is summed in fp32 over key
 // tiles in a fixed descending order (two sums when non-causal, added in a
@@ -50,8 +50,8 @@ struct BwdLayout {
     size_t off = 0;
     L.off_lse2 = off;  off = up256(off + bh * L.npad * 4);
     L.off_dd = off;    off = up256(off + bh * L.npad * 4);
-    L.off_dqacc = off; off = up256(off + 2 * bh * L.npad * (size_t)d * 4);  // lower, upper
-    L.off_cnt = off;   off = up256(off + 2 * bh * L.ntiles * 4);            // lower, upper
+    L.off_dqacc = off; off = up256(off + 2 * bh * L.npad * (size_t)d * 4);  // sums 0, 1
+    L.off_cnt = off;   off = up256(off + 2 * bh * L.ntiles * 4);            // sums 0, 1
     L.off_sched = off; off = up256(off + 16);
     L.total_bytes = off;
     return L;
@@ -78,8 +78,8 @@ struct BwdArgs {
   // Workspace
   float* lse2;   // [B*H, npad] -LSE * log2(e); -inf on rows past the sequence
   float* dd;     // [B*H, npad] D; 0 on rows past the sequence
-  float* dqacc;  // 2 x [B*H, ntiles, d/4, 128, 4] fp32 (lower, upper sums)
-  int* cnt;      // 2 x [B*H, ntiles] dQ ordering counters (lower, upper)
+  float* dqacc;  // 2 x [B*H, ntiles, d/4, 128, 4] fp32 (sum 0, sum 1)
+  int* cnt;      // 2 x [B*H, ntiles] dQ ordering counters (sum 0, sum 1)
   int* sched;    // work counter
   int B, N, H, npad, ntiles;  // N: sequence length (variable length: the longest)
   int d;             // head size (<= D; columns d .. D-1 are zeros from TMA)
@@ -159,9 +159,10 @@ __global__ void __launch_bounds__(256) fa_bwd_dq(const BwdArgs a) {
   const SeqRows seq = seq_rows(a.cu, b, a.N, a.total);
   const int ntile_seq = (seq.len + 127) / 128;
   if (tile >= ntile_seq) return;
-  // Upper sum (key tiles after this query tile): present unless i is the
-  // sequence's last tile.
-  const bool upper = !CAUSAL && tile < ntile_seq - 1;
+  // Sum 1: non-causal, the key tiles after this query tile (none for the
+  // sequence's last tile); causal, the key tiles of odd index (none for
+  // tile 0).
+  const bool upper = CAUSAL ? tile >= 1 : tile < ntile_seq - 1;
   const size_t tile_off = ((size_t)bh * a.ntiles + tile) * 128 * D;  // floats
   const size_t chain = (size_t)a.B * a.H * a.npad * D;               // floats per sum
   const float4* lo = reinterpret_cast<const float4*>(a.dqacc + tile_off);
@@ -286,19 +287,26 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
 // query tile tile(s) = j, j+1, ..., n-1 and then (non-causal only) 0, 1, ...,
 // j-1. Items are handed out head by head, in descending j within a head.
 // Query tile i collects its dQ in two fp32 sums, each over key tiles in
-// descending j: the lower sum (chain 0) from j = i, i-1, ..., 0 and the upper
-// sum (chain 1, non-causal) from j = n-1, n-2, ..., i+1; the contributor with
-// pos(i) = 0 stores, the rest add, each after the previous one has published.
-// fa_bwd_dq adds lower + upper. The contributor a tile waits for (j + 1, same
-// head) was fetched earlier, so the earliest-fetched unfinished item never
-// waits (no deadlock), and it visited that tile one step earlier, so in
-// steady state the wait is already over. (Host-callable too, so these
-// properties are checked on the CPU.)
+// descending j; the contributor with pos(i) = 0 stores, the rest add, each
+// after the previous one has published. fa_bwd_dq adds sum 0 + sum 1.
+//   non-causal: sum 0 (lower) from j = i, i-1, ..., 0 and sum 1 (upper) from
+//     j = n-1, n-2, ..., i+1; a contributor waits for j + 1, which visited
+//     the tile one step earlier.
+//   causal (every key tile j <= i contributes): sum j % 2 from the key tiles
+//     of that parity, j = i or i-1, then two less each time; a contributor
+//     waits for j + 2, which visited the tile two steps earlier, so items
+//     that start together never wait on each other's publication latency.
+// The contributor a tile waits for (same head) was fetched earlier, so the
+// earliest-fetched unfinished item never waits (no deadlock). (Host-callable
+// too, so these properties are checked on the CPU.)
 struct BwdItem {
   int bh, j, T, n;
+  bool causal;
   __host__ __device__ __forceinline__ int tile(int s) const { return j + s < n ? j + s : j + s - n; }
-  __host__ __device__ __forceinline__ int chain(int i) const { return i >= j ? 0 : 1; }
-  __host__ __device__ __forceinline__ int pos(int i) const { return i >= j ? i - j : n - 1 - j; }
+  __host__ __device__ __forceinline__ int chain(int i) const { return causal ? (j & 1) : (i >= j ? 0 : 1); }
+  __host__ __device__ __forceinline__ int pos(int i) const {
+    return causal ? (i - j) >> 1 : (i >= j ? i - j : n - 1 - j);
+  }
 };
 
 // Item number p of a launch over heads of ntiles key tiles each.
@@ -308,6 +316,7 @@ __host__ __device__ __forceinline__ BwdItem decode_item(int p, int ntiles, bool 
   it.j = ntiles - 1 - p % ntiles;  // descending j within a head
   it.n = ntiles;
   it.T = causal ? ntiles - it.j : ntiles;
+  it.causal = causal;
   return it;
 }
 

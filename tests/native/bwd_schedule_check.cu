@@ -8,8 +8,9 @@
 //     0, 1, ..., count-1: one fixed total order, whose first entry stores;
 //  3. the contributor just before (i, j) in that order belongs to an item that
 //     is fetched earlier (smaller item index) and visits tile i one step
-//     earlier in its own sequence, so the earliest unfinished item never
-//     waits and items that start together do not wait on each other.
+//     (non-causal) or two steps (causal) earlier in its own sequence, so the
+//     earliest unfinished item never waits and items that start together do
+//     not wait on each other.
 #include <cstdio>
 #include <cstdlib>
 #include <map>
@@ -65,7 +66,10 @@ int check(int ntiles, int heads, bool causal) {
     for (size_t p = 1; p < v.size(); ++p) {
       const auto& cur = v[by_pos[p]];
       const auto& prev = v[by_pos[p - 1]];
-      if (std::get<1>(prev) >= std::get<1>(cur) || std::get<2>(prev) != std::get<2>(cur) - 1) {
+      // The predecessor is fetched earlier and visits the tile `lag` steps
+      // earlier: one for the non-causal sums, two for the causal parity sums.
+      const int lag = causal ? 2 : 1;
+      if (std::get<1>(prev) >= std::get<1>(cur) || std::get<2>(prev) != std::get<2>(cur) - lag) {
         std::printf("sum (head %d, tile %d): contributor j=%d (item %d, step %d) follows j=%d (item %d, step %d)\n",
                     std::get<0>(kv.first), std::get<1>(kv.first), std::get<3>(cur), std::get<1>(cur), std::get<2>(cur),
                     std::get<3>(prev), std::get<1>(prev), std::get<2>(prev));

@@ -6,7 +6,8 @@ runs it over a range of tile counts, head counts and both masks. It checks that
 every (key tile, query tile) pair is visited once, that each dQ sum's
 contributors form one fixed order starting at position 0, and that each
 contributor's predecessor is fetched earlier and visits the tile one step
-earlier (no deadlock; no waiting between items that start together).
+(non-causal) or two steps (causal) earlier (no deadlock; no waiting between
+items that start together).
 """
 
 import os

@@ -82,6 +82,7 @@ struct BwdArgs {
   int* cnt;      // 2 x [B*H, ntiles] dQ ordering counters (sum 0, sum 1)
   int* sched;    // work counter
   int B, N, H, npad, ntiles;  // N: sequence length (variable length: the longest)
+  int hgroup;        // causal: heads whose items interleave (decode_item)
   int d;             // head size (<= D; columns d .. D-1 are zeros from TMA)
   uint32_t hm;       // head-major tensor maps (kHmQ | kHmK | kHmV | kHmDO | kHmDK | kHmDV)
   Dropout drop;      // used by the DROPOUT instantiation only
@@ -95,8 +96,8 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(256) fa_bwd_prep(const BwdArgs a) {
   // Block (x, bh): rows n = x * kRows + group of head bh, a group of G = D/8
   // lanes per row, 8 elements per lane. Rows of the sequence get
-  // D = rowsum(dO o O) and LSE*log2(e); rows past its end (up to npad) get 0
-  // and +inf (no query: P = 0).
+  // D = rowsum(dO o O) and -LSE*log2(e); rows past its end (up to npad) get 0
+  // and -inf (no query: P = 0).
   constexpr int G = D / 8;
   constexpr int kRows = 256 / G;
   const int bh = blockIdx.y;
@@ -309,11 +310,24 @@ struct BwdItem {
   }
 };
 
-// Item number p of a launch over heads of ntiles key tiles each.
-__host__ __device__ __forceinline__ BwdItem decode_item(int p, int ntiles, bool causal) {
+// Item number p of a launch over heads of ntiles key tiles each. Non-causal
+// (or group = 1): head by head, descending j within a head. Causal: groups of
+// `group` heads, and within a group the k-th item (descending j) of every
+// head before the (k+1)-th of any, so the group's long last items start
+// earlier than head by head and the launch ends on a shorter tail. The host
+// sizes the group so that its heads' Q, dO and dQ sums stay in L2.
+__host__ __device__ __forceinline__ BwdItem decode_item(int p, int ntiles, bool causal, int heads, int group) {
   BwdItem it;
-  it.bh = p / ntiles;
-  it.j = ntiles - 1 - p % ntiles;  // descending j within a head
+  if (causal && group > 1) {
+    const int per_group = group * ntiles;
+    const int g = p / per_group, r = p % per_group;
+    const int gh = heads - g * group < group ? heads - g * group : group;
+    it.bh = g * group + r % gh;
+    it.j = ntiles - 1 - r / gh;
+  } else {
+    it.bh = p / ntiles;
+    it.j = ntiles - 1 - p % ntiles;  // descending j within a head
+  }
   it.n = ntiles;
   it.T = causal ? ntiles - it.j : ntiles;
   it.causal = causal;
@@ -325,7 +339,7 @@ __host__ __device__ __forceinline__ BwdItem decode_item(int p, int ntiles, bool 
 // empty (T = 0) and are skipped by the producer, never handed to the roles.
 template <bool CAUSAL>
 __device__ __forceinline__ BwdItem item_of(const BwdArgs& a, int p, SeqRows* seq) {
-  BwdItem w = decode_item(p, a.ntiles, CAUSAL);
+  BwdItem w = decode_item(p, a.ntiles, CAUSAL, a.B * a.H, a.hgroup);
   *seq = seq_rows(a.cu, w.bh / a.H, a.N, a.total);
   w.n = (seq->len + 127) / 128;
   w.T = w.j < w.n ? (CAUSAL ? w.n - w.j : w.n) : 0;

@@ -1,7 +1,8 @@
 // Host-side check of the backward's work decomposition and dQ ordering, using
 // the kernel header's own decode_item / BwdItem (nothing is launched).
 //
-// For every shape given on the command line (ntiles, heads, causal) it checks:
+// For every shape given on the command line (ntiles, heads, causal, head
+// group) it checks:
 //  1. every (key tile j, query tile i) pair of every head is visited exactly
 //     once (causal: only i >= j);
 //  2. for each (head, query tile, sum), the positions of its contributors are
@@ -19,14 +20,14 @@
 
 #include "../../exact_attention_119_b200/csrc/bwd_kernels.cuh"
 
-int check(int ntiles, int heads, bool causal) {
+int check(int ntiles, int heads, bool causal, int group) {
   // (bh, i, chain) -> list of (pos, item, step, j)
   std::map<std::tuple<int, int, int>, std::vector<std::tuple<int, int, int, int>>> sums;
   std::map<std::tuple<int, int, int>, int> visits;  // (bh, j, i) -> count
   const int total = heads * ntiles;
   for (int item = 0; item < total; ++item) {
-    const fa::BwdItem w = fa::decode_item(item, ntiles, causal);
-    if (w.bh != item / ntiles || w.j < 0 || w.j >= ntiles || w.T < 1 || w.T > ntiles) {
+    const fa::BwdItem w = fa::decode_item(item, ntiles, causal, heads, group);
+    if (w.bh < 0 || w.bh >= heads || w.j < 0 || w.j >= ntiles || w.T < 1 || w.T > ntiles) {
       std::printf("bad item %d: bh %d j %d T %d\n", item, w.bh, w.j, w.T);
       return 1;
     }
@@ -82,10 +83,11 @@ int check(int ntiles, int heads, bool causal) {
 
 int main(int argc, char** argv) {
   int bad = 0, shapes = 0;
-  for (int a = 1; a + 2 < argc; a += 3) {
+  for (int a = 1; a + 3 < argc; a += 4) {
     const int n = std::atoi(argv[a]), h = std::atoi(argv[a + 1]), c = std::atoi(argv[a + 2]);
-    const int r = check(n, h, c != 0);
-    if (r) std::printf("FAILED ntiles %d heads %d causal %d\n", n, h, c);
+    const int g = std::atoi(argv[a + 3]);
+    const int r = check(n, h, c != 0, g);
+    if (r) std::printf("FAILED ntiles %d heads %d causal %d group %d\n", n, h, c, g);
     bad |= r;
     ++shapes;
   }

@@ -37,8 +37,9 @@ def checker(tmp_path_factory):
 def test_items_cover_pairs_once_and_dq_order_is_acyclic(checker, causal):
     args = []
     for ntiles in list(range(1, 41)) + [64, 128, 256]:
-        for heads in (1, 3):
-            args += [str(ntiles), str(heads), str(causal)]
+        for heads in (1, 3, 8, 13, 20):
+            for group in ((1, 2, 8, 16) if causal else (1,)):
+                args += [str(ntiles), str(heads), str(causal), str(group)]
     r = subprocess.run([checker] + args, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stdout[-2000:]
     assert r.stdout.strip().startswith("OK")

@@ -144,6 +144,11 @@ __global__ void __launch_bounds__(256) fa_bwd_prep(const BwdArgs a) {
 // read in their tile-blocked layout (consecutive threads, consecutive rows:
 // coalesced), turned around in shared memory, and each row written with
 // 16-byte stores (consecutive threads, consecutive columns of a row).
+// Invalidate one 128-byte L2 line without writing it back (its data is dead).
+__device__ __forceinline__ void discard_l2(const void* p) {
+  asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
+
 template <int D>
 struct DqCfg {
   static constexpr int kStride = D + 4;  // floats per row in shared memory (bank-conflict padding)
@@ -168,19 +173,37 @@ __global__ void __launch_bounds__(256) fa_bwd_dq(const BwdArgs a) {
   const size_t chain = (size_t)a.B * a.H * a.npad * D;               // floats per sum
   const float4* lo = reinterpret_cast<const float4*>(a.dqacc + tile_off);
   const float4* up = reinterpret_cast<const float4*>(a.dqacc + chain + tile_off);
-  for (int idx = threadIdx.x; idx < 128 * (D / 4); idx += blockDim.x) {
-    const int q = idx / 128, r = idx % 128;  // [D/4][128][4] layout
-    float4 v = lo[idx];
-    if (upper) {
-      const float4 u = up[idx];
-      v.x += u.x;
-      v.y += u.y;
-      v.z += u.z;
-      v.w += u.w;
+  // Every load of the block is issued before the first use (the layout has
+  // 128 * D / 4 float4 per sum, 256 threads).
+  constexpr int kPer = 128 * (D / 4) / 256;
+  float4 v[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) v[k] = lo[threadIdx.x + 256 * k];
+  if (upper) {
+    float4 u[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) u[k] = up[threadIdx.x + 256 * k];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      v[k].x += u[k].x;
+      v[k].y += u[k].y;
+      v[k].z += u[k].z;
+      v[k].w += u[k].w;
     }
-    *reinterpret_cast<float4*>(sm + r * C::kStride + 4 * q) = v;
+  }
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int idx = threadIdx.x + 256 * k;
+    const int q = idx / 128, r = idx % 128;  // [D/4][128][4] layout
+    *reinterpret_cast<float4*>(sm + r * C::kStride + 4 * q) = v[k];
   }
   __syncthreads();
+  // The sums are dead now (the next backward's first contributor stores
+  // before anyone adds): drop their lines from L2 without writing them back.
+  for (int line = threadIdx.x; line < 128 * D * 4 / 128; line += 256) {
+    discard_l2(reinterpret_cast<const char*>(lo) + 128 * line);
+    if (upper) discard_l2(reinterpret_cast<const char*>(up) + 128 * line);
+  }
   for (int idx = threadIdx.x; idx < 128 * (D / 8); idx += blockDim.x) {
     const int r = idx / (D / 8), c8 = idx % (D / 8);
     const int n = tile * 128 + r;

@@ -9,25 +9,26 @@
 //   D_i = rowsum(dO o O)_i,  dS = P o (dP - D),  dK = scale dS^T Q,
 //   dQ = scale dS K.
 //
-// Three launches on the caller's stream:
-//   1. fa_bwd_prep:  D and LSE*log2(e) into padded per-head arrays; zeroes the
-//                    dQ ordering counters and the work counter.
+// Two launches on the caller's stream:
+//   1. fa_bwd_prep:  D and -LSE*log2(e) into padded per-head arrays; zeroes
+//                    the dQ ordering counters and the two work counters.
 //   2. fa_bwd_dkdv:  persistent; one CTA per SM fetches work items (b, h, key
 //                    tile j) from a global counter. Per item K_j, V_j stay in
 //                    shared memory and dK_j, dV_j accumulate in TMEM while
 //                    (Q_i, dO_i) tiles stream through a 2-stage ring. Per
 //                    step, five tcgen05 MMAs: S^T = K Q^T, dP^T = V dO^T,
 //                    dV += P^T dO, dQ_part = dS K, dK += dS^T Q. dQ_part is
-//                    added into fp32 accumulators in a fixed key-tile order
-//                    (per-tile counters say whose turn it is), so the sum is
-//                    deterministic.
-//   3. fa_bwd_dq:    dQ = scale * (sum 0 + sum 1), cast.
+//                    added into two fp32 sums per query tile in a fixed
+//                    key-tile order (per-tile counters say whose turn it
+//                    is), so the sums are deterministic. When the items run
+//                    out, each CTA's dQ warps take finished query tiles from
+//                    a second counter and write dQ = scale * (sum 0 + sum 1).
 //
 // dQ order (BwdItem below). Query tile i's dQ is summed in fp32 over key
-// tiles in a fixed descending order (two sums when non-causal, added in a
-// fixed order at the end), so the result does not depend on scheduling. No
-// wait can deadlock (the earliest-fetched unfinished item waits for nothing),
-// and every wait is bounded anyway.
+// tiles in a fixed descending order (two sums, added in a fixed order at the
+// end), so the result does not depend on scheduling. No wait can deadlock
+// (the earliest-fetched unfinished item waits for nothing, and the finishing
+// of a tile waits only for items), and every wait is bounded anyway.
 #pragma once
 
 #include <algorithm>
@@ -80,7 +81,7 @@ struct BwdArgs {
   float* dd;     // [B*H, npad] D; 0 on rows past the sequence
   float* dqacc;  // 2 x [B*H, ntiles, d/4, 128, 4] fp32 (sum 0, sum 1)
   int* cnt;      // 2 x [B*H, ntiles] dQ ordering counters (sum 0, sum 1)
-  int* sched;    // work counter
+  int* sched;    // [0]: item counter, [1]: counter of query tiles to finish
   int B, N, H, npad, ntiles;  // N: sequence length (variable length: the longest)
   int hgroup;        // causal: heads whose items interleave (decode_item)
   int d;             // head size (<= D; columns d .. D-1 are zeros from TMA)
@@ -134,88 +135,10 @@ __global__ void __launch_bounds__(256) fa_bwd_prep(const BwdArgs a) {
       a.cnt[(size_t)bh * a.ntiles + t] = 0;
       a.cnt[((size_t)a.B * a.H + bh) * a.ntiles + t] = 0;
     }
-    if (bh == 0 && threadIdx.x == 0) *a.sched = 0;
-  }
-}
-
-// ------------------------------------------------------------------ kernel 3
-
-// dQ of one 128-row tile of one head (block (tile, bh)): the fp32 sums are
-// read in their tile-blocked layout (consecutive threads, consecutive rows:
-// coalesced), turned around in shared memory, and each row written with
-// 16-byte stores (consecutive threads, consecutive columns of a row).
-// Invalidate one 128-byte L2 line without writing it back (its data is dead).
-__device__ __forceinline__ void discard_l2(const void* p) {
-  asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
-}
-
-template <int D>
-struct DqCfg {
-  static constexpr int kStride = D + 4;  // floats per row in shared memory (bank-conflict padding)
-  static constexpr int kSmem = 128 * kStride * 4;
-};
-
-template <int D, bool CAUSAL, bool BF16>
-__global__ void __launch_bounds__(256) fa_bwd_dq(const BwdArgs a) {
-  using C = DqCfg<D>;
-  extern __shared__ float4 sm_dq[];
-  float* sm = reinterpret_cast<float*>(sm_dq);
-  const int tile = blockIdx.x, bh = blockIdx.y;
-  const int b = bh / a.H, h = bh % a.H;
-  const SeqRows seq = seq_rows(a.cu, b, a.N, a.total);
-  const int ntile_seq = (seq.len + 127) / 128;
-  if (tile >= ntile_seq) return;
-  // Sum 1: non-causal, the key tiles after this query tile (none for the
-  // sequence's last tile); causal, the key tiles of odd index (none for
-  // tile 0).
-  const bool upper = CAUSAL ? tile >= 1 : tile < ntile_seq - 1;
-  const size_t tile_off = ((size_t)bh * a.ntiles + tile) * 128 * D;  // floats
-  const size_t chain = (size_t)a.B * a.H * a.npad * D;               // floats per sum
-  const float4* lo = reinterpret_cast<const float4*>(a.dqacc + tile_off);
-  const float4* up = reinterpret_cast<const float4*>(a.dqacc + chain + tile_off);
-  // Every load of the block is issued before the first use (the layout has
-  // 128 * D / 4 float4 per sum, 256 threads).
-  constexpr int kPer = 128 * (D / 4) / 256;
-  float4 v[kPer];
-#pragma unroll
-  for (int k = 0; k < kPer; ++k) v[k] = lo[threadIdx.x + 256 * k];
-  if (upper) {
-    float4 u[kPer];
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) u[k] = up[threadIdx.x + 256 * k];
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      v[k].x += u[k].x;
-      v[k].y += u[k].y;
-      v[k].z += u[k].z;
-      v[k].w += u[k].w;
+    if (bh == 0 && threadIdx.x == 0) {
+      a.sched[0] = 0;  // items
+      a.sched[1] = 0;  // query tiles to finish
     }
-  }
-#pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    const int idx = threadIdx.x + 256 * k;
-    const int q = idx / 128, r = idx % 128;  // [D/4][128][4] layout
-    *reinterpret_cast<float4*>(sm + r * C::kStride + 4 * q) = v[k];
-  }
-  __syncthreads();
-  // The sums are dead now (the next backward's first contributor stores
-  // before anyone adds): drop their lines from L2 without writing them back.
-  for (int line = threadIdx.x; line < 128 * D * 4 / 128; line += 256) {
-    discard_l2(reinterpret_cast<const char*>(lo) + 128 * line);
-    if (upper) discard_l2(reinterpret_cast<const char*>(up) + 128 * line);
-  }
-  for (int idx = threadIdx.x; idx < 128 * (D / 8); idx += blockDim.x) {
-    const int r = idx / (D / 8), c8 = idx % (D / 8);
-    const int n = tile * 128 + r;
-    if (n >= seq.len || c8 * 8 >= a.d) continue;
-    const float4 x0 = *reinterpret_cast<const float4*>(sm + r * C::kStride + 8 * c8);
-    const float4 x1 = *reinterpret_cast<const float4*>(sm + r * C::kStride + 8 * c8 + 4);
-    uint4 w;
-    w.x = pack2<BF16>(x0.x * a.scale, x0.y * a.scale);
-    w.y = pack2<BF16>(x0.z * a.scale, x0.w * a.scale);
-    w.z = pack2<BF16>(x1.x * a.scale, x1.y * a.scale);
-    w.w = pack2<BF16>(x1.z * a.scale, x1.w * a.scale);
-    *reinterpret_cast<uint4*>(a.dq + b * a.dq_sb + (seq.row0 + n) * a.dq_sn + h * a.dq_sh + c8 * 8) = w;
   }
 }
 
@@ -274,6 +197,9 @@ struct BwdBarriers {
   int item[2];
   int dq_go;     // the ordering wait succeeded
   int dq_fail;   // some row of the step was not added (sticky)
+  uint64_t fin_turn, fin_done;  // dQ warpgroup, finishing query tiles: tile chosen / tile read
+  int fin_tile;  // the query tile being finished (or past the last one)
+  int fin_ok;    // its sums are complete
   uint32_t tmem_base;
   int abort;
 };
@@ -290,6 +216,10 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
       : "memory");
 }
 
+// Invalidate one 128-byte L2 line without writing it back (its data is dead).
+__device__ __forceinline__ void discard_l2(const void* p) {
+  asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
 __device__ __forceinline__ int ld_acquire(const int* p) {
   int v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -312,7 +242,7 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
 // j-1. Items are handed out head by head, in descending j within a head.
 // Query tile i collects its dQ in two fp32 sums, each over key tiles in
 // descending j; the contributor with pos(i) = 0 stores, the rest add, each
-// after the previous one has published. fa_bwd_dq adds sum 0 + sum 1.
+// after the previous one has published; dQ = scale * (sum 0 + sum 1).
 //   non-causal: sum 0 (lower) from j = i, i-1, ..., 0 and sum 1 (upper) from
 //     j = n-1, n-2, ..., i+1; a contributor waits for j + 1, which visited
 //     the tile one step earlier.
@@ -411,6 +341,8 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(&bars->acc_empty, 256);
     mbar_init(&bars->drain, 1);
     mbar_init(&bars->dq_turn, 1);
+    mbar_init(&bars->fin_turn, 1);
+    mbar_init(&bars->fin_done, 128);
     for (int q = 0; q < 4; ++q) {
       mbar_init(&bars->dq_added[q], 128);
       mbar_init(&bars->dq_rel[q], 1);
@@ -1040,6 +972,105 @@ __global__ void __launch_bounds__(512, 1)
       }
       if (!ok) break;
       ++n_item;
+    }
+    // ---- dQ of finished query tiles. Once the item queue is empty, the
+    // warpgroup takes query tiles from a second counter (head by head, so
+    // the tiles finished first come first), waits until each of the tile's
+    // two sums has all its contributions (its counter reaches the number of
+    // contributors), and writes dQ = scale * (sum 0 + sum 1), added in that
+    // order. The sums are dead afterwards and their L2 lines are dropped
+    // without a write-back. Every contributor was fetched before the queue
+    // ran empty and waits on nothing here, so these waits end.
+    const int total_tiles = a.B * a.H * a.ntiles;
+    const size_t sum_stride = (size_t)a.B * a.H * a.npad * D;  // floats per sum
+    for (int nf = 0; ok; ++nf) {
+      if (threadIdx.x == 256) {
+        const int f = atomicAdd(a.sched + 1, 1);
+        bool go = true;
+        if (f < total_tiles) {
+          const int bh = f / a.ntiles, i = f % a.ntiles;
+          const SeqRows sq = seq_rows(a.cu, bh / a.H, a.N, a.total);
+          const int nt = (sq.len + 127) / 128;
+          if (i < nt) {
+            // Contributors of sum 0 and sum 1 (see BwdItem).
+            const int want0 = CAUSAL ? i / 2 + 1 : i + 1;
+            const int want1 = CAUSAL ? (i + 1) / 2 : nt - 1 - i;
+            const int* c0 = a.cnt + (size_t)bh * a.ntiles + i;
+            const int* c1 = c0 + (size_t)a.B * a.H * a.ntiles;
+            if (ld_acquire(c0) != want0 || ld_acquire(c1) != want1) {
+              const uint64_t t0 = globaltimer();
+              for (uint32_t n = 1;; ++n) {
+                if (ld_acquire(c0) == want0 && ld_acquire(c1) == want1) break;
+                if ((n & 63u) == 0) {
+                  if (*abort) { go = false; break; }
+                  if (globaltimer() - t0 > FA_WAIT_LIMIT_NS) {
+                    record_timeout(2);
+                    *abort = 1;
+                    go = false;
+                    break;
+                  }
+                }
+                __nanosleep(64);
+              }
+            }
+          }
+        }
+        bars->fin_tile = f;
+        bars->fin_ok = go ? 1 : 0;
+        mbar_arrive(&bars->fin_turn);
+      }
+      if (!mbar_wait_warp(&bars->fin_turn, nf & 1, abort)) { ok = false; break; }
+      const int f = bars->fin_tile;
+      if (!bars->fin_ok) { ok = false; break; }
+      if (f >= total_tiles) break;
+      const int bh = f / a.ntiles, i = f % a.ntiles;
+      const int b = bh / a.H, h = bh % a.H;
+      const SeqRows sq = seq_rows(a.cu, b, a.N, a.total);
+      const int nt = (sq.len + 127) / 128;
+      const float* s0 = a.dqacc + ((size_t)bh * a.ntiles + i) * 128 * D;  // [D/4][128][4]
+      const float* s1 = s0 + sum_stride;
+      const bool has1 = CAUSAL ? i >= 1 : i < nt - 1;
+      if (i < nt) {
+        const int n = i * 128 + r;
+        const bool valid = n < sq.len;
+        uint16_t* drow = a.dq + b * a.dq_sb + (sq.row0 + (valid ? n : 0)) * a.dq_sn + h * a.dq_sh;
+#pragma unroll 1
+        for (int q0 = 0; q0 < D / 4; q0 += 8) {
+          float4 x[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) x[k] = __ldcg(reinterpret_cast<const float4*>(s0) + (q0 + k) * 128 + r);
+          if (has1) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const float4 u = __ldcg(reinterpret_cast<const float4*>(s1) + (q0 + k) * 128 + r);
+              x[k].x += u.x;
+              x[k].y += u.y;
+              x[k].z += u.z;
+              x[k].w += u.w;
+            }
+          }
+          if (valid) {
+#pragma unroll
+            for (int k = 0; k < 8; k += 2) {
+              const int col = (q0 + k) * 4;
+              if (col < a.d)
+                *reinterpret_cast<uint4*>(drow + col) = make_uint4(
+                    pack2<BF16>(x[k].x * a.scale, x[k].y * a.scale), pack2<BF16>(x[k].z * a.scale, x[k].w * a.scale),
+                    pack2<BF16>(x[k + 1].x * a.scale, x[k + 1].y * a.scale),
+                    pack2<BF16>(x[k + 1].z * a.scale, x[k + 1].w * a.scale));
+            }
+          }
+        }
+      }
+      // Every row of the tile has been read: drop the sums' lines.
+      mbar_arrive(&bars->fin_done);
+      if (!mbar_wait_warp(&bars->fin_done, nf & 1, abort)) { ok = false; break; }
+      if (i < nt) {
+        for (int line = r; line < 4 * D; line += 128) {
+          discard_l2(reinterpret_cast<const char*>(s0) + 128 * line);
+          if (has1) discard_l2(reinterpret_cast<const char*>(s1) + 128 * line);
+        }
+      }
     }
   }
 

@@ -428,8 +428,8 @@ fa_status run_fwd(const Problem& p, const void* q, const void* k, const void* v,
 
 // ----------------------------------------------------------------- backward
 
-// The three backward launches on one stream: preprocessing, the persistent
-// dK/dV (and dQ partial) kernel, and the dQ cast.
+// The two backward launches on one stream: preprocessing, and the
+// persistent dK/dV kernel (which also sums, scales and casts dQ).
 // Tensor maps of the backward: inputs q, k, v, dout and outputs dk, dv.
 struct BwdMaps {
   CUtensorMap q, k, v, dout, dk, dv;
@@ -460,13 +460,7 @@ cudaError_t launch_bwd_t(const BwdMaps& m, const BwdArgs& a, int sms, cudaStream
     set_detail_cuda("cudaEventRecord(profile end)", e);
     return e;
   }
-  auto dqk = fa_bwd_dq<D, CAUSAL, BF16>;
-  e = set_smem(dqk, DqCfg<D>::kSmem);
-  if (e != cudaSuccess) {
-    set_detail_cuda("cudaFuncSetAttribute(fa_bwd_dq)", e);
-    return e;
-  }
-  return launch("fa_bwd_dq", dqk, dim3(a.ntiles, a.B * a.H), 256, DqCfg<D>::kSmem, s, 1, a);
+  return cudaSuccess;
 }
 
 template <int D, bool DROPOUT>

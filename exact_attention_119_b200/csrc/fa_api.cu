@@ -723,9 +723,9 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   cudaError_t e = cudaSuccess;
   uint8_t* scratch = noalloc_scratch(&e);
   if (scratch == nullptr) return FA_ERR_CUDA;
-  // The preprocessing launch rewrites D and LSE*log2(e), zeroes the ordering
-  // counters and the work counter; the first key tile stores (not adds) each
-  // dQ tile. Nothing left in the scratch by an earlier call is read.
+  // The preprocessing launch rewrites D and -LSE*log2(e), zeroes the ordering
+  // counters and both work counters; the first contributor of each dQ sum
+  // stores (not adds). Nothing left in the scratch by an earlier call is read.
   return run_bwd(p, q, k, v, o, dout, lse, dq, dk, dv, scratch, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -263,6 +263,13 @@ struct BwdItem {
   }
 };
 
+// Number of key tiles that add into sum c of query tile i of a head with nt
+// key tiles (the finishing step waits for this many publications).
+__host__ __device__ __forceinline__ int sum_contributors(int i, int nt, bool causal, int c) {
+  if (causal) return c == 0 ? i / 2 + 1 : (i + 1) / 2;  // even / odd j <= i
+  return c == 0 ? i + 1 : nt - 1 - i;                   // j <= i / j > i
+}
+
 // Item number p of a launch over heads of ntiles key tiles each. Non-causal
 // (or group = 1): head by head, descending j within a head. Causal: groups of
 // `group` heads, and within a group the k-th item (descending j) of every
@@ -992,9 +999,8 @@ __global__ void __launch_bounds__(512, 1)
           const SeqRows sq = seq_rows(a.cu, bh / a.H, a.N, a.total);
           const int nt = (sq.len + 127) / 128;
           if (i < nt) {
-            // Contributors of sum 0 and sum 1 (see BwdItem).
-            const int want0 = CAUSAL ? i / 2 + 1 : i + 1;
-            const int want1 = CAUSAL ? (i + 1) / 2 : nt - 1 - i;
+            const int want0 = sum_contributors(i, nt, CAUSAL, 0);
+            const int want1 = sum_contributors(i, nt, CAUSAL, 1);
             const int* c0 = a.cnt + (size_t)bh * a.ntiles + i;
             const int* c1 = c0 + (size_t)a.B * a.H * a.ntiles;
             if (ld_acquire(c0) != want0 || ld_acquire(c1) != want1) {
@@ -1029,7 +1035,7 @@ __global__ void __launch_bounds__(512, 1)
       const int nt = (sq.len + 127) / 128;
       const float* s0 = a.dqacc + ((size_t)bh * a.ntiles + i) * 128 * D;  // [D/4][128][4]
       const float* s1 = s0 + sum_stride;
-      const bool has1 = CAUSAL ? i >= 1 : i < nt - 1;
+      const bool has1 = sum_contributors(i, nt, CAUSAL, 1) > 0;
       if (i < nt) {
         const int n = i * 128 + r;
         const bool valid = n < sq.len;

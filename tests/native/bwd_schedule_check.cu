@@ -11,7 +11,9 @@
 //     is fetched earlier (smaller item index) and visits tile i one step
 //     (non-causal) or two steps (causal) earlier in its own sequence, so the
 //     earliest unfinished item never waits and items that start together do
-//     not wait on each other.
+//     not wait on each other;
+//  4. sum_contributors (the counts the finishing step waits for) equals the
+//     number of contributors of every sum, empty sums included.
 #include <cstdio>
 #include <cstdlib>
 #include <map>
@@ -49,6 +51,19 @@ int check(int ntiles, int heads, bool causal, int group) {
         const int got = it == visits.end() ? 0 : it->second;
         if (got != want) {
           std::printf("head %d pair (i %d, j %d) visited %d times\n", bh, i, j, got);
+          return 1;
+        }
+      }
+  // 4. the finishing step's contributor counts match the sums, including the
+  //    empty ones.
+  for (int bh = 0; bh < heads; ++bh)
+    for (int i = 0; i < ntiles; ++i)
+      for (int c = 0; c < 2; ++c) {
+        const auto it = sums.find({bh, i, c});
+        const int got = it == sums.end() ? 0 : (int)it->second.size();
+        if (got != fa::sum_contributors(i, ntiles, causal, c)) {
+          std::printf("head %d tile %d sum %d: %d contributors, finishing step expects %d\n", bh, i, c, got,
+                      fa::sum_contributors(i, ntiles, causal, c));
           return 1;
         }
       }

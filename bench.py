@@ -614,7 +614,8 @@ def main():
             "roofline": {"bound": "tensor", "kernel": "fa_bwd_dkdv", "achieved": dkdv_tflops / world, "peak": peak,
                          "unit": "TFLOP/s", "frac": dkdv_tflops / world / peak, "traffic": traffic,
                          "note": ("the backward's dK/dV kernel, which runs all five backward contractions "
-                                  "(10*B*H*N^2*d, halved when causal), timed by events on its own launch; "
+                                  "(10*B*H*N^2*d, halved when causal) and then sums and casts dQ, timed by "
+                                  "events on its own launch; "
                                   f"peak {peak_kind}; traffic: {traffic_note}")},
             "kernels": {
                 "fa_fwd_kernel": {"tflops": fwd_tflops / world, "frac": fwd_tflops / world / peak,

@@ -89,6 +89,28 @@ def test_head_major_inputs_and_strided_outputs(causal):
 
 
 @pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d,dtype", [(128, "bf16"), (64, "fp16")])
+def test_head_major_outputs(d, dtype, causal):
+    # O, dQ, dK, dV written into [B, H, N, d] storage through [B, N, H, d]
+    # views: the output tensor maps are head-major, and N = 300 leaves a
+    # ragged last tile whose rows past N must not be written.
+    import exact_attention_119_b200 as fa
+    B, N, H = 2, 300, 3
+    case = Case(B, N, H, d, dtype, causal, seed=47)
+    q, k, v, do = (case.torch(n) for n in ("q", "k", "v", "do"))
+    store = [torch.full((B, H, N + 8, d), 7.0, dtype=q.dtype, device="cuda") for _ in range(4)]
+    out, dq, dk, dv = (t[:, :, :N].transpose(1, 2) for t in store)
+    assert out.stride() == (H * (N + 8) * d, d, (N + 8) * d, 1)
+    o, lse = fa.forward(q, k, v, case.scale, causal, out=out)
+    grads = fa.backward(q, k, v, o, do, lse, case.scale, causal, dq, dk, dv)
+    assert fa.check_device_status() == 0
+    check_fwd(o, lse, case)
+    check_grads(grads, case)
+    for t in store:
+        assert torch.all(t[:, :, N:] == 7.0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("d", [8, 16, 32, 40, 48, 72, 80, 96, 112, 120])
 def test_head_sizes(d, causal):
     # Head sizes between the kernels' 64- and 128-column tiles: the tensor
